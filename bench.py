@@ -1,0 +1,342 @@
+"""Benchmark of the NVFP4 W4A4 linear (quantize + GEMM) on Qwen3-8B-shaped
+prefill projections at 8192 tokens: QKV (4096 -> 6144), O (4096 -> 4096),
+gate/up (4096 -> 24576), down (12288 -> 4096).
+
+One step = the four projections, each: tensor scale of X, NVFP4 quantization
+of X, block-scaled FP4 GEMM against the pre-quantized weight (weights are
+quantized once, outside the timed region).  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (plain C + numpy binary64) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_w4a4_quantized_03_b200 import inputs  # noqa: E402
+
+TOKENS = 8192
+METRIC = "W4A4 NVFP4 linear TFLOPS (quant+GEMM) & % of B200 FP4 peak; quant GB/s"
+WORKLOAD = "qwen3-8b prefill projections (qkv, o, gate_up, down) at 8192 tokens, NVFP4 W4A4"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            flags = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                     "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+            while not self._stop.is_set():
+                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, bit in flags.items():
+                    if r & bit:
+                        self.reasons.add(name)
+                time.sleep(self.period)
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.reasons.add(f"nvml-unavailable: {type(e).__name__}")
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _projection_inputs(seed_base: int, device):
+    projs = []
+    for i, p in enumerate(inputs.QWEN3_8B_PROJECTIONS):
+        x = inputs.activation_bf16(TOKENS, p.K, seed=seed_base + i, outlier_channels=inputs.outlier_count(p.K),
+                                   outlier_scale=50.0, device=device)
+        w = inputs.weight_bf16(p.N, p.K, seed=seed_base + 100 + i, device=device)
+        projs.append((p, x, w))
+    return projs
+
+
+def _flops_per_step():
+    return sum(2.0 * TOKENS * p.N * p.K for p in inputs.QWEN3_8B_PROJECTIONS)
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample_step(projs_cpu, rows_per_proj: int, rng):
+    """One oracle pass over a sample: alpha of the whole X, then quantize,
+    dequantize and binary64-multiply `rows_per_proj` sampled rows against the
+    pre-dequantized weight.  Returns the sampled FLOPs."""
+    import oracle
+    flops = 0.0
+    for p, xb, w_hat in projs_cpu:
+        ax = oracle.tensor_scale(xb)
+        rows = np.sort(rng.choice(xb.shape[0], rows_per_proj, replace=False))
+        xc, xs = oracle.quantize(np.ascontiguousarray(xb[rows]), ax)
+        y = oracle.bf16_rne_array(oracle.gemm_f64(oracle.dequantize(xc, xs, ax), w_hat))
+        assert y.shape == (rows_per_proj, p.N)
+        flops += 2.0 * rows_per_proj * p.N * p.K
+    return flops
+
+
+def _oracle_projections():
+    import oracle
+    out = []
+    for p, x, w in _projection_inputs(0, "cpu"):
+        xb, wb = inputs.bf16_bits(x), inputs.bf16_bits(w)
+        aw = oracle.tensor_scale(wb)
+        wc, ws = oracle.quantize(wb, aw)
+        out.append((p, xb, oracle.dequantize(wc, ws, aw)))
+    return out
+
+
+def cpu_baseline(target_s: float = 12.0):
+    import oracle
+    projs = _oracle_projections()
+    rng = np.random.default_rng(0)
+    rows = 32
+    oracle_sample_step(projs, 8, rng)                      # warm-up
+    t0 = time.perf_counter()
+    flops, steps = 0.0, 0
+    while time.perf_counter() - t0 < target_s or steps < 2:
+        flops += oracle_sample_step(projs, rows, rng)
+        steps += 1
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{steps} oracle steps, each {rows} of {TOKENS} rows per projection (alpha over all rows), "
+                      f"weights dequantized once beforehand; {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    projs = _oracle_projections()
+    rng = np.random.default_rng(0)
+    rows = 8
+    for _ in range(args.warmup):
+        oracle_sample_step(projs, rows, rng)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += oracle_sample_step(projs, rows, rng)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "tokens": TOKENS},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"each step: {rows} of {TOKENS} rows per projection"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU path
+
+def run_ours(args, world, rank, local):
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+
+    projs = _projection_inputs(rank * 1000, device)
+    work = []
+    for p, x, w in projs:
+        qw = mq.quantize(w)                       # offline weight quantization (not timed)
+        qx = mq.QuantizedTensor(TOKENS, p.K, device)
+        ws = mq.workspace(mq.mq_workspace_bytes(), device)
+        y = torch.empty(TOKENS, p.N, dtype=torch.bfloat16, device=device)
+        work.append(dict(p=p, x=x, qw=qw, qx=qx, ws=ws, y=y))
+        del w
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        for i, t in enumerate(work):
+            p = t["p"]
+            mq.mq_tensor_scale(t["x"], t["qx"].alpha, t["ws"], stream)
+            mq.mq_nvfp4_quantize(t["x"], t["qx"].alpha, t["qx"].codes, t["qx"].scales, stream)
+            if ev is not None:
+                ev[i][0].record(stream)
+            mq.mq_nvfp4_gemm(t["qx"].codes, t["qx"].scales, t["qx"].alpha, t["qw"].codes, t["qw"].scales,
+                             t["qw"].alpha, TOKENS, p.N, p.K, t["y"], t["ws"], stream)
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for t in work:
+        assert mq.mq_read_status(t["ws"]) == mq.MQ_OK
+
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in work] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        end.record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    elapsed_ms = _max_over_ranks(start.elapsed_time(end), world, device)
+    gemm_ms = sum(e[0].elapsed_time(e[1]) for ev in evs for e in ev) / args.steps
+    for t in work:
+        assert mq.mq_read_status(t["ws"]) == mq.MQ_OK
+
+    flops = _flops_per_step()
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
+
+    # end to end through the public API with host buffers
+    e2e = _e2e(args, work, device, stream)
+
+    peaks, peaks_src = _peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]        # nominal fp4 : bf16 = 9 : 2.25
+    gemm_tflops = flops / (gemm_ms / 1e3) / 1e12
+    # quantizer bandwidth: 2 B read (amax) + 2 B read + 0.5625 B written per X element
+    x_elems = sum(TOKENS * t["p"].K for t in work)
+    quant_ms = ms_per_step - gemm_ms
+    quant_gbs = x_elems * (2.0 + 2.5625) / (quant_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": TOKENS, "parallelism": f"replicas{world}",
+                   "l2": "no flush: per-step working set ~1.1 GB (bf16 X 384 MB, FP4 W 92 MB, bf16 Y 608 MB) > 126 MB L2"},
+        "fp4_frac_of_nominal_9pf": value / 9000.0,
+        "quant_gbs": quant_gbs,
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp4_peak, "traffic": None,
+                     "kernel": "mq::gemm::k_gemm", "peak_source": f"{peaks_src}: 4 x bf16_tflops_sustained"},
+        "gpu_launches": 12 * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _e2e(args, work, device, stream):
+    """Pinned host X -> device, mq_linear_w4a4, device -> pinned host Y, per step."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    host_x = [t["x"].cpu().pin_memory() for t in work]
+    host_y = [torch.empty(t["y"].shape, dtype=torch.bfloat16).pin_memory() for t in work]
+    dx = [torch.empty_like(t["x"]) for t in work]
+    lws = [mq.workspace(mq.mq_linear_w4a4_workspace_bytes(TOKENS, t["p"].K), device) for t in work]
+
+    def step():
+        for i, t in enumerate(work):
+            dx[i].copy_(host_x[i], non_blocking=True)
+            mq.mq_linear_w4a4(dx[i], t["qw"].codes, t["qw"].scales, t["qw"].alpha, t["p"].N, t["y"], lws[i], stream)
+            host_y[i].copy_(t["y"], non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    h2d = sum(h.numel() * 2 for h in host_x)
+    d2h = sum(h.numel() * 2 for h in host_y)
+    return {"value": _flops_per_step() / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    world, rank, local = _dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * mq.h -- C ABI of libmq.so: NVFP4 W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The method (NVFP4 two-level microscaling, weights and activations both in
+ * 4-bit E2M1, W4A4) is the one stated in
+ *   "Mix-Quant：面向智能体LLM的量化预填充与精确解码" (paper.rainbus.top digest),
+ *   section 方法步骤详情, step (3), and section NVFP4 微缩放量化; and
+ *   "Mix-Quant: Quantized Prefilling, Precise Decoding for Agentic LLMs"
+ *   (r9-hu paper digest), section Method, item 1:
+ *
+ *     sigma_b = Pi_E4M3( max_{i in b} |x_i| / (alpha_x * q_max) )   (block scale)
+ *     q_i     = Pi_FP4 ( x_i / (alpha_x * sigma_b(i)) )            (element code)
+ *     xhat_i  = alpha_x * sigma_b(i) * q_i                          (dequantized value)
+ *
+ * with blocks b of 16 consecutive elements along K, q_max = 6, round to
+ * nearest.  The arithmetic the kernels use where the pages leave it open:
+ *     alpha_x = fl32(amax / 2688)      (amax = max |x| over the tensor; 1 if amax = 0)
+ *     sigma_b = RNE_E4M3_satfinite( fl32( amax_b / fl32(6 * alpha_x) ) )
+ *     q_i     = RNE_E2M1_satfinite( fl32( x_i * fl32( 1 / fl32(alpha_x * sigma_b) ) ) )
+ *     q_i     = +0 for every element of a block whose sigma_b is 0
+ *     Y       = bf16_RNE( fl32(alpha_a * alpha_b) * fp32 tensor-core sum_k (sigma q)_a (sigma q)_b )
+ *
+ * Data layout (all row-major, K contiguous; the nn.Linear layout W[N, K]):
+ *   bf16 tensors : [rows, K], 2 bytes per element.
+ *   codes        : [rows, K/2] bytes; element 2j in the low nibble of byte j,
+ *                  E2M1 code = sign(bit 3) | exponent(bits 2..1) | mantissa(bit 0).
+ *   scales       : E4M3 (OCP E4M3FN) bytes in the order the Blackwell
+ *                  block-scaled MMA reads: atoms of 128 rows x 4 scale columns
+ *                  (512 bytes), atom (row/128, kblock/4) at byte
+ *                  ((row/128) * ceil(K/64) + kblock/4) * 512; inside an atom
+ *                  (row, kblock) sits at (row%32)*16 + ((row/32)%4)*4 + kblock%4.
+ *                  Rows are padded to a multiple of 128 (padding bytes are 0).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller owns
+ *     every buffer.  The library never allocates or frees memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only
+ *     enqueue work; they return before it runs.
+ *   - The return value is an mq_status.  A synchronous error (bad argument,
+ *     shape, alignment, device) enqueues nothing.  Errors found on the device
+ *     (a bounded wait that expired) are written to the workspace status word,
+ *     read back with mq_read_status.
+ *   - Shapes: rows, M, N >= 1; K >= 64 and K % 64 == 0.  Base pointers must be
+ *     16-byte aligned.  Inputs are finite bf16: NaN/Inf are outside the
+ *     contract (alpha becomes NaN, nothing else is guaranteed).
+ *   - Device: compute capability 10.0 (B200), else MQ_ERR_ARCH.
+ */
+#ifndef MQ_H
+#define MQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mq_status {
+    MQ_OK = 0,
+    MQ_ERR_INVALID_ARG = -1,   /* null pointer or bad size argument            */
+    MQ_ERR_SHAPE = -2,         /* K not a positive multiple of 64, M/N <= 0      */
+    MQ_ERR_ALIGN = -3,         /* a base pointer is not 16-byte aligned          */
+    MQ_ERR_ARCH = -4,          /* current device is not compute capability 10.0  */
+    MQ_ERR_WORKSPACE = -5,     /* workspace missing or smaller than required     */
+    MQ_ERR_CUDA = -6,          /* a CUDA runtime call failed                     */
+    MQ_ERR_TIMEOUT = -7        /* device side: a bounded wait expired            */
+} mq_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mq_status_string(int status);
+
+/* Bytes of packed E2M1 codes for a [rows, K] tensor: rows * K / 2. */
+size_t mq_nvfp4_codes_bytes(int64_t rows, int64_t K);
+
+/* Bytes of the block-scale buffer for a [rows, K] tensor in the MMA order:
+ * ceil(rows/128)*128 * ceil(K/64)*4. */
+size_t mq_nvfp4_scales_bytes(int64_t rows, int64_t K);
+
+/* Bytes of workspace mq_tensor_scale and mq_nvfp4_gemm use (a 256-byte header
+ * holding the amax accumulator, a block counter and the status word). */
+size_t mq_workspace_bytes(void);
+
+/* Bytes of workspace mq_linear_w4a4 needs for an [M, K] activation: the
+ * header plus room for the quantized activation (codes and scales). */
+size_t mq_linear_w4a4_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * Tensor-level scale alpha_x of a bf16 tensor ("张量级尺度", section NVFP4
+ * 微缩放量化 of the paper.rainbus.top digest; alpha_x in the r9-hu digest,
+ * section Method, item 1):  *alpha = fl32(max|x| / 2688), or 1 if max|x| = 0.
+ *   x      : device, numel bf16 values (16-byte aligned)
+ *   alpha  : device, 1 float, written
+ *   ws     : device workspace of >= mq_workspace_bytes() bytes, zero-filled
+ *            before its first use; every call leaves its counters at zero.
+ *            Calls that share a workspace must not overlap on the GPU.
+ */
+int mq_tensor_scale(const void *x, int64_t numel, float *alpha, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * NVFP4 quantization of a bf16 [rows, K] tensor with a given alpha_x
+ * (block scale sigma_b and element codes q_i as above; section 方法步骤详情,
+ * step (3); section Method, item 1).
+ *   x      : device bf16 [rows, K]
+ *   alpha  : device, 1 float (e.g. written by mq_tensor_scale)
+ *   codes  : device, mq_nvfp4_codes_bytes(rows, K) bytes, written
+ *   scales : device, mq_nvfp4_scales_bytes(rows, K) bytes, written (padding = 0)
+ */
+int mq_nvfp4_quantize(const void *x, int64_t rows, int64_t K, const float *alpha,
+                      uint8_t *codes, uint8_t *scales, void *stream);
+
+/*
+ * Block-scaled FP4 GEMM on two quantized operands (W4A4: both sides NVFP4,
+ * section 方法步骤详情, step (3)):
+ *   y[m, n] = bf16( fl32(alpha_a * alpha_b) * sum_k (sigma q)_a[m, k] (sigma q)_b[n, k] )
+ *   a_codes/a_scales : A = [M, K] (activations), alpha_a device float
+ *   b_codes/b_scales : B = [N, K] (weights, nn.Linear layout), alpha_b device float
+ *   y                : device bf16 [M, N], written
+ *   ws               : optional (may be NULL) workspace of >= mq_workspace_bytes()
+ *                      bytes; when given, a timeout is reported in its status word.
+ * Tensor cores accumulate in fp32; the result matches the exact product of
+ * the dequantized operands rounded to bf16 to within about 1e-3 relative
+ * Frobenius error.
+ */
+int mq_nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *alpha_a,
+                  const uint8_t *b_codes, const uint8_t *b_scales, const float *alpha_b,
+                  int64_t M, int64_t N, int64_t K, void *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The W4A4 linear layer of the FP4 prefill path: Y = X W^T with X quantized
+ * on the fly (alpha_x from X, then codes and scales) and W quantized offline
+ * (mq_tensor_scale + mq_nvfp4_quantize on W).
+ *   x        : device bf16 [M, K]
+ *   w_codes, w_scales, alpha_w : quantized W [N, K]
+ *   y        : device bf16 [M, N], written
+ *   ws       : device workspace of >= mq_linear_w4a4_workspace_bytes(M, K)
+ *              bytes, zero-filled before its first use; calls sharing it
+ *              must not overlap on the GPU.
+ * Y equals mq_nvfp4_gemm applied to (mq_tensor_scale, mq_nvfp4_quantize)(X)
+ * and W bit for bit.
+ */
+int mq_linear_w4a4(const void *x, int64_t M, int64_t K,
+                   const uint8_t *w_codes, const uint8_t *w_scales, const float *alpha_w, int64_t N,
+                   void *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronizes `stream`, then reads the status word of a workspace into
+ * *device_status (MQ_OK or MQ_ERR_TIMEOUT) and clears it.  `ws` is a device
+ * pointer, `device_status` a host pointer.
+ */
+int mq_read_status(void *ws, void *stream, int32_t *device_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MQ_H */

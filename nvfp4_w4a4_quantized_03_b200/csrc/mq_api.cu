@@ -1,0 +1,185 @@
+// mq_api.cu -- the extern "C" boundary of libmq.so (declared in include/mq.h):
+// argument validation, per-device attribute cache, and the launches.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mq.h"
+#include "mq_internal.h"
+
+namespace {
+
+constexpr long long DEFAULT_TIMEOUT_CYCLES = 4000000000LL;   // ~2-3 s of SM clock
+constexpr int MAX_DEVICES = 64;
+
+struct DeviceInfo {
+    int checked = 0;
+    int ok = 0;
+    int num_sms = 0;
+};
+DeviceInfo g_dev[MAX_DEVICES];
+std::mutex g_mu;
+
+int current_device_info(int* num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MQ_ERR_CUDA;
+        d.ok = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        d.checked = 1;
+    }
+    if (!d.ok) return MQ_ERR_ARCH;
+    *num_sms = d.num_sms;
+    return MQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+int check_rows_k(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0 || K % 64 != 0) return MQ_ERR_SHAPE;
+    if (rows > (int64_t)1 << 31 || K > (int64_t)1 << 24) return MQ_ERR_SHAPE;
+    return MQ_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mq_status_string(int status) {
+    switch (status) {
+        case MQ_OK: return "MQ_OK";
+        case MQ_ERR_INVALID_ARG: return "MQ_ERR_INVALID_ARG";
+        case MQ_ERR_SHAPE: return "MQ_ERR_SHAPE";
+        case MQ_ERR_ALIGN: return "MQ_ERR_ALIGN";
+        case MQ_ERR_ARCH: return "MQ_ERR_ARCH";
+        case MQ_ERR_WORKSPACE: return "MQ_ERR_WORKSPACE";
+        case MQ_ERR_CUDA: return "MQ_ERR_CUDA";
+        case MQ_ERR_TIMEOUT: return "MQ_ERR_TIMEOUT";
+        default: return "MQ_ERR_UNKNOWN";
+    }
+}
+
+size_t mq_nvfp4_codes_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 0;
+    return (size_t)rows * (size_t)(K / 2);
+}
+
+size_t mq_nvfp4_scales_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 0;
+    return (size_t)mq::padded_rows(rows) * (size_t)mq::scale_atom_cols(K) * 4;
+}
+
+size_t mq_workspace_bytes(void) { return mq::WS_HEADER_BYTES; }
+
+size_t mq_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0) return 0;
+    return mq::WS_HEADER_BYTES + round256(mq_nvfp4_codes_bytes(M, K)) + round256(mq_nvfp4_scales_bytes(M, K));
+}
+
+int mq_tensor_scale(const void* x, int64_t numel, float* alpha, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !alpha || numel <= 0) return MQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < mq::WS_HEADER_BYTES) return MQ_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(alpha) & 3u)) return MQ_ERR_ALIGN;
+    int sms = 0;
+    int st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_amax(x, numel, static_cast<uint32_t*>(ws), alpha, sms,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int mq_nvfp4_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
+                      uint8_t* scales, void* stream) {
+    if (!x || !alpha || !codes || !scales) return MQ_ERR_INVALID_ARG;
+    int st = check_rows_k(rows, K);
+    if (st != MQ_OK) return st;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(alpha) & 3u))
+        return MQ_ERR_ALIGN;
+    int sms = 0;
+    st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_quantize(x, rows, K, alpha, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
+static int gemm_checked(const uint8_t* a_codes, const uint8_t* a_scales, const float* alpha_a,
+                        const uint8_t* b_codes, const uint8_t* b_scales, const float* alpha_b, int64_t M,
+                        int64_t N, int64_t K, void* y, int* status, cudaStream_t stream) {
+    if (!a_codes || !a_scales || !alpha_a || !b_codes || !b_scales || !alpha_b || !y) return MQ_ERR_INVALID_ARG;
+    int st = check_rows_k(M, K);
+    if (st != MQ_OK) return st;
+    st = check_rows_k(N, K);
+    if (st != MQ_OK) return st;
+    if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
+        !aligned16(y))
+        return MQ_ERR_ALIGN;
+    int sms = 0;
+    st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    mq::GemmArgs g{a_codes, a_scales, alpha_a, b_codes, b_scales, alpha_b, y, M, N, K,
+                   status, DEFAULT_TIMEOUT_CYCLES, 0};
+    return cuda_status(mq::launch_gemm(g, sms, stream));
+}
+
+int mq_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* alpha_a, const uint8_t* b_codes,
+                  const uint8_t* b_scales, const float* alpha_b, int64_t M, int64_t N, int64_t K, void* y,
+                  void* ws, size_t ws_bytes, void* stream) {
+    int* status = nullptr;
+    if (ws) {
+        if (ws_bytes < mq::WS_HEADER_BYTES) return MQ_ERR_WORKSPACE;
+        if (!aligned16(ws)) return MQ_ERR_ALIGN;
+        status = static_cast<int*>(ws) + mq::WS_STATUS;
+    }
+    return gemm_checked(a_codes, a_scales, alpha_a, b_codes, b_scales, alpha_b, M, N, K, y, status,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int mq_linear_w4a4(const void* x, int64_t M, int64_t K, const uint8_t* w_codes, const uint8_t* w_scales,
+                   const float* alpha_w, int64_t N, void* y, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !w_codes || !w_scales || !alpha_w || !y) return MQ_ERR_INVALID_ARG;
+    int st = check_rows_k(M, K);
+    if (st != MQ_OK) return st;
+    st = check_rows_k(N, K);
+    if (st != MQ_OK) return st;
+    if (!ws || ws_bytes < mq_linear_w4a4_workspace_bytes(M, K)) return MQ_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned256(ws) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
+        return MQ_ERR_ALIGN;
+    int sms = 0;
+    st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* words = static_cast<uint32_t*>(ws);
+    float* alpha_x = reinterpret_cast<float*>(words + mq::WS_ALPHA);
+    uint8_t* x_codes = static_cast<uint8_t*>(ws) + mq::WS_HEADER_BYTES;
+    uint8_t* x_scales = x_codes + round256(mq_nvfp4_codes_bytes(M, K));
+    cudaError_t e = mq::launch_amax(x, M * K, words, alpha_x, sms, s);
+    if (e == cudaSuccess) e = mq::launch_quantize(x, M, K, alpha_x, x_codes, x_scales, s);
+    if (e != cudaSuccess) return MQ_ERR_CUDA;
+    mq::GemmArgs g{x_codes, x_scales, alpha_x, w_codes, w_scales, alpha_w, y, M, N, K,
+                   reinterpret_cast<int*>(words + mq::WS_STATUS), DEFAULT_TIMEOUT_CYCLES, 0};
+    return cuda_status(mq::launch_gemm(g, sms, s));
+}
+
+int mq_read_status(void* ws, void* stream, int32_t* device_status) {
+    if (!ws || !device_status) return MQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* word = static_cast<int32_t*>(ws) + mq::WS_STATUS;
+    int32_t v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MQ_ERR_CUDA;
+    if (cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MQ_ERR_CUDA;
+    if (cudaMemset(word, 0, sizeof v) != cudaSuccess) return MQ_ERR_CUDA;
+    *device_status = v;
+    return MQ_OK;
+}
+
+}  // extern "C"

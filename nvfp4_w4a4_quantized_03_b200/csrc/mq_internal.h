@@ -1,0 +1,46 @@
+// mq_internal.h -- declarations shared by the CUDA translation units of
+// libmq.so (not part of the public C ABI, which is include/mq.h).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mq {
+
+// Workspace header, in 32-bit words.  Every kernel that uses it leaves the
+// counters at zero when it finishes, so a zero-filled header stays valid.
+enum WsWord : int {
+    WS_AMAX_BITS = 0,   // running max of |x| as a bf16 bit pattern (u32)
+    WS_TICKET = 1,      // blocks of the amax pass that have finished
+    WS_STATUS = 2,      // device-side status (0 = ok, else an mq_status code)
+    WS_ALPHA = 3,       // alpha_x written by the amax pass of mq_linear_w4a4
+};
+constexpr size_t WS_HEADER_BYTES = 256;
+
+// Scale storage: atoms of 128 rows x 4 scale columns (512 bytes), ordered
+// row-tile major, k-tile minor (the order the block-scaled MMA reads).
+__host__ __device__ inline int64_t scale_atom_cols(int64_t K) { return (K / 16 + 3) / 4; }
+__host__ __device__ inline int64_t padded_rows(int64_t rows) { return (rows + 127) / 128 * 128; }
+
+// Launchers (enqueue on `stream`, no synchronisation).
+cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
+                        int num_sms, cudaStream_t stream);
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
+                            uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+
+struct GemmArgs {
+    const uint8_t* a_codes;
+    const uint8_t* a_scales;
+    const float* alpha_a;
+    const uint8_t* b_codes;
+    const uint8_t* b_scales;
+    const float* alpha_b;
+    void* y;
+    int64_t M, N, K;
+    int* status;            // may be null
+    long long timeout_cycles;
+    int fault_skip_first_load;   // failure-detection tests only
+};
+cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
+
+}  // namespace mq

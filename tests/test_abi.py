@@ -1,0 +1,69 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/mq.h declares; host-side argument checks answer without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(mq_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def libmq():
+    from nvfp4_w4a4_quantized_03_b200 import build, mq
+    build.build()
+    return mq.lib()
+
+
+def test_header_declares_the_path():
+    names = set(_declared_functions())
+    for required in ("mq_tensor_scale", "mq_nvfp4_quantize", "mq_nvfp4_gemm", "mq_linear_w4a4"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(libmq):
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    out = subprocess.run(["nm", "-D", "--defined-only", mq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(mq_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in _declared_functions():
+        getattr(libmq, n)
+
+
+def test_sizes(libmq):
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    assert mq.mq_nvfp4_codes_bytes(8192, 4096) == 8192 * 2048
+    assert mq.mq_nvfp4_scales_bytes(8192, 4096) == 8192 * 256
+    assert mq.mq_nvfp4_scales_bytes(1, 64) == 128 * 4
+    assert mq.mq_nvfp4_scales_bytes(130, 320) == 256 * 20
+    assert mq.mq_workspace_bytes() == 256
+    assert mq.mq_linear_w4a4_workspace_bytes(128, 1024) == 256 + 65536 + 8192
+
+
+def test_host_validation_without_gpu(libmq):
+    """Bad arguments are refused before any device call."""
+    vp = ctypes.c_void_p
+    p16 = vp(4096)          # an aligned dummy address; never dereferenced
+    assert libmq.mq_nvfp4_quantize(p16, 128, 100, p16, p16, p16, None) == -2      # K % 64
+    assert libmq.mq_nvfp4_quantize(p16, 0, 128, p16, p16, p16, None) == -2        # rows
+    assert libmq.mq_nvfp4_quantize(None, 1, 64, p16, p16, p16, None) == -1        # null
+    assert libmq.mq_nvfp4_quantize(vp(4097), 1, 64, p16, p16, p16, None) == -3    # misaligned
+    assert libmq.mq_tensor_scale(p16, 64, p16, p16, 16, None) == -5                # workspace too small
+    assert libmq.mq_linear_w4a4(p16, 128, 1024, p16, p16, p16, 256, p16, p16, 1024, None) == -5
+    assert libmq.mq_nvfp4_gemm(p16, p16, p16, p16, p16, p16, 1, 1, 96, p16, None, 0, None) == -2
+    assert libmq.mq_status_string(-7) == b"MQ_ERR_TIMEOUT"

@@ -1,0 +1,131 @@
+"""GPU parity of the block-scaled FP4 GEMM (mq_nvfp4_gemm) and of the fused
+linear (mq_linear_w4a4) against the CPU oracle.
+
+Y = bf16(xhat . what^T), xhat = alpha sigma q ("Mix-Quant：面向智能体LLM的量化预填充
+与精确解码", section 方法步骤详情, step (3); W4A4).  Tolerance: relative
+Frobenius error <= 1e-3 against the oracle's bf16 result on the same quantized
+operands; bit-exact where every partial sum is exact in binary32.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_w4a4_quantized_03_b200 import inputs, mq
+from tests.gpu_helpers import bf16_bits_to_f64, bits, dev, gpu_quantize, rel_frobenius
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+
+
+def _gemm(qa, qb, M, N, K):
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev())
+    ws = mq.workspace(mq.mq_workspace_bytes(), dev())
+    mq.mq_nvfp4_gemm(qa.codes, qa.scales, qa.alpha, qb.codes, qb.scales, qb.alpha, M, N, K, y, ws)
+    torch.cuda.synchronize()
+    assert mq.mq_read_status(ws) == mq.MQ_OK
+    return bits(y)
+
+
+def _upload(codes_np, logical_scales, K, alpha):
+    rows = codes_np.shape[0]
+    q = mq.QuantizedTensor(rows, K, dev())
+    q.codes.copy_(torch.from_numpy(np.ascontiguousarray(codes_np).reshape(-1)))
+    q.scales.copy_(torch.from_numpy(oracle.scales_to_stored(logical_scales, K)))
+    q.alpha.fill_(alpha)
+    return q
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (128, 256, 256), (200, 300, 512), (1, 8, 64), (257, 513, 320)])
+def test_exact_products_bit_exact(M, N, K):
+    """Codes random, scales powers of two in [2^-2, 2^2], alpha = 1: every
+    partial sum is exact in binary32, so Y must equal the oracle bit for bit.
+    Pins the MMA's reading of code nibbles, E4M3 scales and the scale order."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    pow2 = np.array([(e + 7) << 3 for e in range(-2, 3)], np.uint8)   # E4M3 codes of 2^e
+    ac = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    bc = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    asc = pow2[rng.integers(0, 5, size=(M, K // 16))]
+    bsc = pow2[rng.integers(0, 5, size=(N, K // 16))]
+    y = _gemm(_upload(ac, asc, K, 1.0), _upload(bc, bsc, K, 1.0), M, N, K)
+    ref = oracle.bf16_rne_array(oracle.gemm_f64(oracle.dequantize(ac, asc, 1.0), oracle.dequantize(bc, bsc, 1.0)))
+    bad = np.argwhere(y != ref)
+    assert len(bad) == 0, f"{len(bad)} mismatches, first {bad[:4].tolist()}"
+
+
+def test_alpha_product_scaling():
+    """alpha_a * alpha_b (powers of two) scales Y exactly."""
+    M, N, K = 128, 256, 128
+    rng = np.random.default_rng(3)
+    ac = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    bc = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sc = np.full((M, K // 16), 0x38, np.uint8)   # 1.0
+    sb = np.full((N, K // 16), 0x38, np.uint8)
+    y = _gemm(_upload(ac, sc, K, 2.0 ** -3), _upload(bc, sb, K, 2.0 ** 5), M, N, K)
+    ref = oracle.bf16_rne_array(4.0 * oracle.gemm_f64(oracle.dequantize(ac, sc, 1.0), oracle.dequantize(bc, sb, 1.0)))
+    assert np.array_equal(y, ref)
+
+
+def _random_case(M, N, K, seed, student_t=False):
+    if student_t:
+        x = inputs.student_t_activation_bf16(M, K, seed=seed)
+    else:
+        x = inputs.activation_bf16(M, K, seed=seed, outlier_channels=max(1, inputs.outlier_count(K)),
+                                   outlier_scale=50.0)
+    w = inputs.weight_bf16(N, K, seed=seed + 1000)
+    return x, w
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 1024, 1024), (1, 256, 64), (3, 17, 128), (17, 3, 64), (130, 300, 320),
+                                   (257, 513, 1024), (300, 257, 128), (512, 1024, 4096), (96, 4096, 12288)])
+def test_gemm_random_against_oracle(M, N, K):
+    x, w = _random_case(M, N, K, seed=M + N + K)
+    ax, xc, xs, qx = gpu_quantize(x)
+    aw, wc, wsc, qw = gpu_quantize(w)
+    y = _gemm(qx, qw, M, N, K)
+    ref = oracle.linear_w4a4(bits(x), bits(w))
+    assert ref["alpha_x"] == ax and ref["alpha_w"] == aw
+    assert np.array_equal(ref["x_codes"], xc) and np.array_equal(ref["w_codes"], wc)
+    err = rel_frobenius(bf16_bits_to_f64(y), bf16_bits_to_f64(ref["y_bf16"]))
+    assert err <= TOL, err
+
+
+def test_linear_equals_separate_calls_and_oracle():
+    M, N, K = 200, 768, 1024
+    x, w = _random_case(M, N, K, seed=5, student_t=True)
+    qw = mq.quantize(w.to(dev()))
+    _, _, _, qx = gpu_quantize(x)
+    y_sep = _gemm(qx, qw, M, N, K)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev())
+    ws = mq.workspace(mq.mq_linear_w4a4_workspace_bytes(M, K), dev())
+    for _ in range(2):      # the workspace is reusable call after call
+        mq.mq_linear_w4a4(x.to(dev()), qw.codes, qw.scales, qw.alpha, N, y, ws)
+        torch.cuda.synchronize()
+        assert mq.mq_read_status(ws) == mq.MQ_OK
+        assert np.array_equal(bits(y), y_sep)
+    ref = oracle.linear_w4a4(bits(x), bits(w))
+    assert rel_frobenius(bf16_bits_to_f64(bits(y)), bf16_bits_to_f64(ref["y_bf16"])) <= TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("proj", inputs.QWEN3_8B_PROJECTIONS, ids=lambda p: p.name)
+def test_prefill_projection_8k_sampled_rows(proj):
+    """Full 8192-token projections through mq_linear_w4a4; the oracle checks
+    alpha on the whole activation and 256 sampled output rows in full."""
+    M, K, N = 8192, proj.K, proj.N
+    x, w = _random_case(M, N, K, seed=17)
+    lin = mq.LinearW4A4(w.to(dev()))
+    y = lin(x.to(dev()))
+    torch.cuda.synchronize()
+    assert mq.mq_read_status(lin._ws) == mq.MQ_OK
+    xb, wb = bits(x), bits(w)
+    ax = oracle.tensor_scale(xb)
+    aw = oracle.tensor_scale(wb)
+    assert float(lin.w.alpha.item()) == aw
+    rows = np.sort(np.random.default_rng(0).choice(M, 256, replace=False))
+    xc, xs = oracle.quantize(np.ascontiguousarray(xb[rows]), ax)
+    wc, wsc = oracle.quantize(wb, aw)
+    y64 = oracle.gemm_f64(oracle.dequantize(xc, xs, ax), oracle.dequantize(wc, wsc, aw))
+    ref = oracle.bf16_rne_array(y64)
+    got = bits(y)[rows]
+    assert rel_frobenius(bf16_bits_to_f64(got), bf16_bits_to_f64(ref)) <= TOL
