@@ -1,0 +1,45 @@
+"""The multi-rank host path of bench.py on CPU: two gloo ranks, the timing
+reduction takes the maximum over ranks and every rank takes the same
+collective steps (replicas, no data-path collective)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    import bench
+    w, r, _ = bench._dist()
+    assert (w, r) == (world, rank)
+    bench._barrier(w)
+    mx = bench._max_over_ranks(10.0 + rank, w, "cpu")
+    bench._barrier(w)
+    q.put((rank, mx))
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_over_ranks():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    assert got == [(0, 11.0), (1, 11.0)]
