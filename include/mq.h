@@ -143,6 +143,33 @@ int mq_linear_w4a4(const void *x, int64_t M, int64_t K,
                    void *y, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * mq_linear_w4a4 for callers that cannot allocate device memory -- for
+ * example a plugin inside a host application that owns all device memory and
+ * hands extensions no allocator, or C code that must not call cudaMalloc
+ * because it synchronizes the device.  The paper has no counterpart: this is a
+ * deployment convenience of this library, not a step of the method.
+ *
+ * Same arguments and result as mq_linear_w4a4, without the workspace: the
+ * library uses its own scratch, one static device array of
+ * MQ_NOALLOC_SCRATCH_BYTES (64 MiB) that every GPU loading libmq.so holds
+ * until the process exits.  Nothing is allocated or freed by this call.
+ *   - Shapes whose mq_linear_w4a4_workspace_bytes(M, K) exceeds
+ *     MQ_NOALLOC_SCRATCH_BYTES are refused with MQ_ERR_WORKSPACE (e.g.
+ *     M = 8192 with K up to 12288 fits; M = 131072, K = 4096 does not).
+ *   - The first call on a device looks up the scratch's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one scratch: calls whose GPU work overlaps (other
+ *     streams, other host threads) race and corrupt each other's results;
+ *     serialize them.  Each call clears the scratch header before use.
+ *   - Device-side timeouts land in the scratch's status word, which the caller
+ *     cannot read; use mq_linear_w4a4 with a workspace to observe them.
+ */
+#define MQ_NOALLOC_SCRATCH_BYTES (64u << 20)
+int mq_linear_w4a4_noalloc(const void *x, int64_t M, int64_t K,
+                           const uint8_t *w_codes, const uint8_t *w_scales, const float *alpha_w, int64_t N,
+                           void *y, void *stream);
+
+/*
  * Synchronizes `stream`, then reads the status word of a workspace into
  * *device_status (MQ_OK or MQ_ERR_TIMEOUT) and clears it.  `ws` is a device
  * pointer, `device_status` a host pointer.

@@ -185,3 +185,22 @@ class LinearW4A4:
             out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         mq_linear_w4a4(x, self.w.codes, self.w.scales, self.w.alpha, self.N, out, self._ws, stream)
         return out
+
+
+# -- the allocation-free variant (library-owned scratch) ---------------------
+
+MQ_NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def mq_linear_w4a4_noalloc(x: torch.Tensor, w_codes, w_scales, alpha_w, N: int, y: torch.Tensor,
+                           stream=None) -> None:
+    """mq_linear_w4a4 without a workspace, for callers that cannot allocate:
+    the library's static 64 MiB scratch is used (shared by every call on a
+    device, so calls must not overlap on the GPU)."""
+    f = lib().mq_linear_w4a4_noalloc
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    f.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
+    f.restype = ctypes.c_int
+    M, K = x.shape
+    _check(f(_ptr(x), M, K, _ptr(w_codes), _ptr(w_scales), _ptr(alpha_w), N, _ptr(y), _stream(stream)),
+           "mq_linear_w4a4_noalloc")
