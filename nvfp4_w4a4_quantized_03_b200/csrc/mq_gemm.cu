@@ -11,14 +11,19 @@
 // Design (one CTA per SM, persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer: A/B code tiles (128-byte swizzle) and the two
 //               scale tiles (plain bulk copies) into a 4-stage ring.
-//   warp 1      allocates TMEM; one lane issues tcgen05.cp (scales -> TMEM)
-//               and tcgen05.mma (K = 64 per instruction, 4 per stage), then
-//               tcgen05.commit to release stages and to publish a tile.
-//   warps 2..9  epilogue: tcgen05.ld the 128 x 256 fp32 accumulator, scale by
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (K = 64 per
+//               instruction, 4 per stage) and tcgen05.commit to release
+//               stages and to publish a finished tile.
+//   warps 2..5  scale writers: move each stage's block scales from shared
+//               memory into that stage's TMEM scale columns with tcgen05.st,
+//               one warp per 32-lane TMEM sub-partition (the MMA reads the
+//               scales replicated in all four).  Done off the MMA thread,
+//               this costs the tensor pipe nothing, where tcgen05.cp from the
+//               MMA thread measured ~45 cycles per copy, serialised with the
+//               MMAs.
+//   warps 6..13 epilogue: drain the 128 x 256 fp32 accumulator from TMEM into
+//               registers, release it to the MMA warp, then scale by
 //               alpha_a * alpha_b, round to bf16 and store.
-// Every wait on an mbarrier is bounded; on a timeout the kernel records
-// MQ_ERR_TIMEOUT in the status word, unwinds every role, waits (bounded) for
-// its own copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "mq_internal.h"
@@ -38,16 +43,20 @@ constexpr int B_BYTES = BN * BK / 2;          // 32 KiB
 constexpr int SFA_BYTES = BM * BK / 16;       // 2 KiB
 constexpr int SFB_BYTES = BN * BK / 16;       // 4 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SF_WARPS = 4;
 constexpr int EPI_WARPS = 8;
-constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr int FIRST_SF_WARP = 2;
+constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + SF_WARPS;
+constexpr int THREADS = (FIRST_EPI_WARP + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SFA_COL = BN;                    // 4 columns per MMA
-constexpr uint32_t SFB_COL = SFA_COL + 4 * NKB;     // 8 columns per MMA
+constexpr uint32_t SF_COLS_PER_STAGE = 12 * NKB;    // per MMA: A 4 columns, B 8 columns
+constexpr uint32_t SF_COL = BN;                     // stage st: SF_COL + st * SF_COLS_PER_STAGE
+constexpr uint32_t SFB_OFF = 4 * NKB;               // B scales after the A scales of a stage
 constexpr int GROUP_M = 16;                         // tile raster: M-blocks per group
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
-static_assert(SFB_COL + 8 * NKB <= TMEM_COLS, "TMEM budget");
+static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM budget");
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
 
 // Instruction descriptor of kind::mxf4nvf4: E2M1 x E2M1, UE4M3 scales,
@@ -72,8 +81,9 @@ struct Params {
 };
 
 struct Smem {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[STAGES];       // TMA bytes of a stage landed
+    uint64_t sf_ready[STAGES];   // the stage's scales are in TMEM
+    uint64_t empty[STAGES];      // the stage's MMAs completed
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -111,6 +121,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&s->full[i], 1);
+            mbar_init(&s->sf_ready[i], SF_WARPS);
             mbar_init(&s->empty[i], 1);
         }
         mbar_init(&s->acc_full, 1);
@@ -192,7 +203,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < p.k_stages; ++kt) {
-                    if (!mbar_wait_bounded(&s->full[st], phase, p.timeout, abort_flag)) {
+                    // the stage's data is in shared memory and its scales in TMEM
+                    if (!mbar_wait_bounded(&s->sf_ready[st], phase, p.timeout, abort_flag)) {
                         raise_abort(s, p);
                         ok = false;
                         break;
@@ -200,16 +212,12 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     tc_fence_after();
                     const int nkb = min(NKB, p.kblocks - kt * NKB);
                     const uint32_t a0 = smem_u32(stage_a(st)), b0 = smem_u32(stage_b(st));
-                    const uint32_t sfa0 = smem_u32(stage_sfa(st)), sfb0 = smem_u32(stage_sfb(st));
+                    const uint32_t sf = tmem + SF_COL + st * SF_COLS_PER_STAGE;
                     for (int kb = 0; kb < nkb; ++kb) {
-                        tmem_cp_32x128b_x4(tmem + SFA_COL + kb * 4, smem_desc(sfa0 + kb * 512, 16, 128, 0));
-                        tmem_cp_32x128b_x4(tmem + SFB_COL + kb * 8, smem_desc(sfb0 + kb * 512, 16, 128, 0));
-                        tmem_cp_32x128b_x4(tmem + SFB_COL + kb * 8 + 4,
-                                           smem_desc(sfb0 + SFB_BYTES / 2 + kb * 512, 16, 128, 0));
                         const uint64_t ad = smem_desc(a0 + kb * (MMA_K / 2), 16, 1024, 2);
                         const uint64_t bd = smem_desc(b0 + kb * (MMA_K / 2), 16, 1024, 2);
-                        mma_mxf4nvf4(tmem + ACC_COL, ad, bd, IDESC, tmem + SFA_COL + kb * 4,
-                                     tmem + SFB_COL + kb * 8, (kt | kb) != 0);
+                        mma_mxf4nvf4(tmem + ACC_COL, ad, bd, IDESC, sf + kb * 4, sf + SFB_OFF + kb * 8,
+                                     (kt | kb) != 0);
                     }
                     mma_commit(&s->empty[st]);
                     if (++st == STAGES) { st = 0; phase ^= 1; }
@@ -222,10 +230,44 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             mma_commit(&s->drain);
             mbar_wait_bounded(&s->drain, 0, p.timeout, nullptr);
         }
+    } else if (warp < FIRST_EPI_WARP) {
+        // ------------------------------------------------------------ scale writers
+        // Lane l of the warp owning TMEM sub-partition q writes row l of each
+        // 512-byte scale atom (16 bytes: rows l, l+32, l+64, l+96 of the tile,
+        // 4 scales each) into 4 consecutive columns of TMEM lane 32q + l.
+        const int quad = warp & 3;
+        int st = 0;
+        uint32_t phase = 0;
+        for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
+            bool ok = true;
+            for (int kt = 0; kt < p.k_stages; ++kt) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s->full[st], phase, p.timeout, abort_flag));
+                if (!ok) break;
+                const int nkb = min(NKB, p.kblocks - kt * NKB);
+                const uint8_t* sfa = stage_sfa(st) + lane * 16;
+                const uint8_t* sfb = stage_sfb(st) + lane * 16;
+                const uint32_t t = tmem + ((uint32_t)(quad * 32) << 16) + SF_COL + st * SF_COLS_PER_STAGE;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    tmem_st_32x32b_x4(t + kb * 4, *reinterpret_cast<const uint4*>(sfa + kb * 512));
+                    tmem_st_32x32b_x4(t + SFB_OFF + kb * 8, *reinterpret_cast<const uint4*>(sfb + kb * 512));
+                    tmem_st_32x32b_x4(t + SFB_OFF + kb * 8 + 4,
+                                      *reinterpret_cast<const uint4*>(sfb + SFB_BYTES / 2 + kb * 512));
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s->sf_ready[st]);
+                if (++st == STAGES) { st = 0; phase ^= 1; }
+            }
+            if (!ok) {
+                if (lane == 0) raise_abort(s, p);
+                break;
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int quad = warp & 3;                  // TMEM lanes this warp may read
-        const int half = (warp - 2) / 4;            // which 128 accumulator columns
+        const int quad = warp & 3;                          // TMEM lanes this warp may read
+        const int half = (warp - FIRST_EPI_WARP) / 4;       // which 128 accumulator columns
         const float ab = __fmul_rn(__ldg(p.alpha_a), __ldg(p.alpha_b));
         const bool vec_ok = (p.N % 8) == 0;
         uint32_t acc_phase = 0;
@@ -242,33 +284,55 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             tc_fence_after();
             const int row = mb * BM + quad * 32 + lane;
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(taddr + c * 32, r);
-                tmem_ld_wait();
-                if (c == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s->acc_empty);
-                }
-                const int col0 = nb * BN + half * 128 + c * 32;
-                if (row < p.M && col0 < p.N) {
-                    uint32_t packed[16];
+            const int colh = nb * BN + half * 128;
+            if (vec_ok && nb * BN + BN <= p.N) {
+                // Whole tile inside Y: drain this warp's 32 x 128 block of the
+                // accumulator (scaled and rounded to bf16 on the way), hand TMEM
+                // back so the next tile's MMAs overlap the stores, then store.
+                uint32_t packed[4][16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        packed[j] = cvt_bf16x2(__fmul_rn(__uint_as_float(r[2 * j + 1]), ab),
-                                               __fmul_rn(__uint_as_float(r[2 * j]), ab));
-                    __nv_bfloat16* dst = p.y + (int64_t)row * p.N + col0;
-                    if (vec_ok && col0 + 32 <= p.N) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
+                        packed[c][j] = cvt_bf16x2(__fmul_rn(__uint_as_float(r[2 * j + 1]), ab),
+                                                  __fmul_rn(__uint_as_float(r[2 * j]), ab));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s->acc_empty);
+                if (row < p.M) {
+                    uint4* d4 = reinterpret_cast<uint4*>(p.y + (int64_t)row * p.N + colh);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                    } else {
-                        uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+                            d4[c * 4 + j] = make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
+                                                       packed[c][4 * j + 2], packed[c][4 * j + 3]);
+                }
+            } else {
+                // Ragged right edge (or N not a multiple of 8): one 32-column
+                // chunk at a time, element stores past the last full chunk.
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tmem_ld_wait();
+                    if (c == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s->acc_empty);
+                    }
+                    const int col0 = colh + c * 32;
+                    if (row >= p.M || col0 >= p.N) continue;
+                    uint16_t* d16 = reinterpret_cast<uint16_t*>(p.y + (int64_t)row * p.N + col0);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) d16[j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
+                    for (int j = 0; j < 32; ++j) {
+                        if (col0 + j < p.N) {
+                            const uint32_t two = cvt_bf16x2(0.0f, __fmul_rn(__uint_as_float(r[j]), ab));
+                            d16[j] = (uint16_t)(two & 0xffffu);
+                        }
                     }
                 }
             }
