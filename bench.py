@@ -248,6 +248,10 @@ def run_ours(args, world, rank, local):
     _barrier(world)
     elapsed_ms = _max_over_ranks(start.elapsed_time(end), world, device)
     gemm_ms = sum(e[0].elapsed_time(e[1]) for ev in evs for e in ev) / args.steps
+    by_proj = {}
+    for i, t in enumerate(work):
+        ms_i = sum(ev[i][0].elapsed_time(ev[i][1]) for ev in evs) / args.steps
+        by_proj[t["p"].name] = 2.0 * TOKENS * t["p"].N * t["p"].K / (ms_i / 1e3) / 1e12
     for t in work:
         assert mq.mq_read_status(t["ws"]) == mq.MQ_OK
 
@@ -272,6 +276,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": WORKLOAD, "tokens": TOKENS, "parallelism": f"replicas{world}",
                    "l2": "no flush: per-step working set ~1.1 GB (bf16 X 384 MB, FP4 W 92 MB, bf16 Y 608 MB) > 126 MB L2"},
         "fp4_frac_of_nominal_9pf": value / 9000.0,
+        "gemm_tflops_by_projection": by_proj,
         "quant_gbs": quant_gbs,
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp4_peak, "traffic": None,

@@ -8,23 +8,41 @@
 // fp32 by the tensor cores.  A is [M, K] and B is [N, K], both K-major (the
 // nn.Linear layout), codes packed two per byte, scales in the MMA layout.
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: A/B code tiles (128-byte swizzle) and the two
-//               scale tiles (plain bulk copies) into a 4-stage ring.
-//   warp 1      allocates TMEM; one lane issues tcgen05.mma (K = 64 per
-//               instruction, 4 per stage) and tcgen05.commit to release
-//               stages and to publish a finished tile.
+// Design: persistent warp-specialised kernel, one CTA per SM, in two forms.
+//   PAIR = 1   one CTA computes a 128 x 256 output tile (cta_group::1 MMA).
+//   PAIR = 2   a cluster of two CTAs computes a 256 x 256 tile: each CTA
+//              stages its own 128 rows of A and its own 128 rows of B, the
+//              even CTA issues cta_group::2 MMAs that read both CTAs' shared
+//              memory and accumulate 128 rows in each CTA's TMEM.  Per SM
+//              this halves B's shared-memory reads and cuts L2 traffic by a
+//              third against PAIR = 1.
+// Warp roles (both forms):
+//   warp 0      producer: per stage, the block-scale tiles (plain bulk copies,
+//               completing on this CTA's sf_full) and then the A/B code tiles
+//               (TMA, 128-byte swizzle; in the pair form both CTAs' copies
+//               complete on CTA 0's `ready` barrier).
+//   warp 1      allocates TMEM; in the (even) CTA one lane issues
+//               tcgen05.mma (K = 64 per instruction, 4 per stage) and
+//               tcgen05.commit to release stages and to publish a tile.
 //   warps 2..5  scale writers: move each stage's block scales from shared
-//               memory into that stage's TMEM scale columns with tcgen05.st,
+//               memory into that stage's TMEM scale columns with tcgen05.st
+//               and arrive on CTA 0's `ready` barrier (one barrier per stage
+//               is all the MMA thread waits on),
 //               one warp per 32-lane TMEM sub-partition (the MMA reads the
-//               scales replicated in all four).  Done off the MMA thread,
-//               this costs the tensor pipe nothing, where tcgen05.cp from the
+//               scales replicated in all four).  Done off the MMA thread this
+//               costs the tensor pipe nothing, where tcgen05.cp issued by the
 //               MMA thread measured ~45 cycles per copy, serialised with the
 //               MMAs.
-//   warps 6..13 epilogue: drain the 128 x 256 fp32 accumulator from TMEM into
-//               registers, release it to the MMA warp, then scale by
-//               alpha_a * alpha_b, round to bf16 and store.
+//   warps 6..13 epilogue: drain the CTA's 128 x 256 fp32 accumulator into
+//               registers (scaled by alpha_a * alpha_b, rounded to bf16),
+//               release it to the MMA thread, then store.
+// Every wait on an mbarrier is bounded; on a timeout the kernel records
+// MQ_ERR_TIMEOUT in the status word, unwinds every role, waits (bounded) for
+// its own copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstdlib>
 
 #include "mq_internal.h"
 #include "mq_ptx.cuh"
@@ -32,17 +50,9 @@
 namespace mq {
 namespace gemm {
 
-constexpr int BM = 128;               // rows of A per tile (TMEM lanes)
-constexpr int BN = 256;               // rows of B per tile (accumulator columns)
-constexpr int BK = 256;               // K elements per pipeline stage
+constexpr int BM = 128;               // A rows per CTA (TMEM lanes)
+constexpr int BN = 256;               // accumulator columns (N of one MMA)
 constexpr int MMA_K = 64;             // K elements per tcgen05.mma (kind::mxf4nvf4)
-constexpr int NKB = BK / MMA_K;       // MMAs per stage
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK / 2;          // 16 KiB
-constexpr int B_BYTES = BN * BK / 2;          // 32 KiB
-constexpr int SFA_BYTES = BM * BK / 16;       // 2 KiB
-constexpr int SFB_BYTES = BN * BK / 16;       // 4 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int SF_WARPS = 4;
 constexpr int EPI_WARPS = 8;
 constexpr int FIRST_SF_WARP = 2;
@@ -50,22 +60,47 @@ constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + SF_WARPS;
 constexpr int THREADS = (FIRST_EPI_WARP + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COLS_PER_STAGE = 12 * NKB;    // per MMA: A 4 columns, B 8 columns
 constexpr uint32_t SF_COL = BN;                     // stage st: SF_COL + st * SF_COLS_PER_STAGE
-constexpr uint32_t SFB_OFF = 4 * NKB;               // B scales after the A scales of a stage
-constexpr int GROUP_M = 16;                         // tile raster: M-blocks per group
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int GROUP_M = 8;                          // tile raster: M-blocks per group
+constexpr int MAX_STAGES = 10;
+constexpr int BARRIER_BYTES = 512;
+constexpr int SMEM_LIMIT = 232448;                  // dynamic shared memory per block on sm_100
 
-static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM budget");
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
-
-// Instruction descriptor of kind::mxf4nvf4: E2M1 x E2M1, UE4M3 scales,
-// K-major A and B, M = 128, N = 256, dense K = 64.
-constexpr uint32_t IDESC = (1u << 7)              // A format E2M1
-                         | (1u << 10)             // B format E2M1
-                         | ((uint32_t)(BN >> 3) << 17)
-                         | (0u << 23)             // scale format UE4M3
-                         | ((uint32_t)(BM >> 4) << 24);
+// PAIR: CTAs per output tile (1 or 2).  BK: K elements per pipeline stage
+// (128 or 256; the code tiles use the 64- or 128-byte swizzle).
+template <int PAIR, int BK>
+struct Cfg {
+    static constexpr int NKB = BK / MMA_K;                    // MMAs per stage
+    static constexpr int ROW_BYTES = BK / 2;                  // bytes of one code row per stage
+    static constexpr int A_BYTES = BM * ROW_BYTES;
+    static constexpr int B_ROWS = BN / PAIR;                  // B rows staged by one CTA
+    static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
+    static constexpr int SFA_BYTES = BM * BK / 16;
+    static constexpr int SFB_BYTES = BN * BK / 16;            // scales of all 256 B rows
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr uint32_t SF_COLS_PER_STAGE = 12 * NKB;   // per MMA: A 4 columns, B 8 columns
+    static constexpr uint32_t SFB_OFF = 4 * NKB;              // B scales after the A scales of a stage
+    static constexpr int SMEM_STAGES = (SMEM_LIMIT - 1024 - BARRIER_BYTES) / STAGE_BYTES;
+    static constexpr int TMEM_STAGES = (TMEM_COLS - SF_COL) / SF_COLS_PER_STAGE;
+    static constexpr int STAGES = SMEM_STAGES < TMEM_STAGES ? (SMEM_STAGES < MAX_STAGES ? SMEM_STAGES : MAX_STAGES)
+                                                            : (TMEM_STAGES < MAX_STAGES ? TMEM_STAGES : MAX_STAGES);
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + BARRIER_BYTES;
+    static constexpr int TILE_M = BM * PAIR;
+    static constexpr uint32_t SWIZZLE = ROW_BYTES == 128 ? 2 : 4;     // descriptor layout: 128B / 64B swizzle
+    static constexpr uint32_t SBO = 8 * ROW_BYTES;                    // 8-row swizzle atom
+    // Instruction descriptor of kind::mxf4nvf4: E2M1 x E2M1, UE4M3 scales,
+    // K-major A and B, M = TILE_M, N = 256, dense K = 64.
+    static constexpr uint32_t IDESC = (1u << 7)            // A format E2M1
+                                    | (1u << 10)           // B format E2M1
+                                    | ((uint32_t)(BN >> 3) << 17)
+                                    | (0u << 23)           // scale format UE4M3
+                                    | ((uint32_t)(TILE_M >> 4) << 24);
+    static_assert(BK == 128 || BK == 256, "stage depth");
+    static_assert(STAGES >= 2 && STAGES <= MAX_STAGES, "stage count");
+    static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM budget");
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the swizzle atoms");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
+};
 
 struct Params {
     const uint8_t* a_scales;
@@ -74,16 +109,18 @@ struct Params {
     const float* alpha_b;
     __nv_bfloat16* y;
     int M, N, K;
-    int m_blocks, n_blocks, tiles, k_stages, kblocks, katoms, b_row_tiles;
+    int m_blocks, n_blocks, tiles, k_stages, kblocks, katoms, a_row_tiles, b_row_tiles;
     int* status;
     long long timeout;
     int fault_skip_first_load;
 };
 
 struct Smem {
-    uint64_t full[STAGES];       // TMA bytes of a stage landed
-    uint64_t sf_ready[STAGES];   // the stage's scales are in TMEM
-    uint64_t empty[STAGES];      // the stage's MMAs completed
+    // ready[s] (used in CTA 0): the stage's A and B codes landed in both CTAs
+    // (TMA bytes) and every scale writer put its scales into TMEM (arrivals)
+    uint64_t ready[MAX_STAGES];
+    uint64_t sf_full[MAX_STAGES];    // this CTA's block scales of a stage landed
+    uint64_t empty[MAX_STAGES];      // the stage's MMAs completed
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
@@ -105,27 +142,52 @@ __device__ __forceinline__ void raise_abort(Smem* s, const Params& p) {
     if (p.status) atomicExch(p.status, -7 /* MQ_ERR_TIMEOUT */);
 }
 
+// Arrive on a barrier of the even CTA of the pair (or on the local one).
+template <int PAIR>
+__device__ __forceinline__ void arrive_leader(uint64_t* bar) {
+    if (PAIR == 2) mbar_arrive_remote(mapa_shared(smem_u32(bar), 0));
+    else mbar_arrive(bar);
+}
+
+template <int PAIR>
+__device__ __forceinline__ void commit_to_all(uint64_t* bar) {
+    if (PAIR == 2) mma_commit_pair_mc(bar, 0x3);
+    else mma_commit(bar);
+}
+
+template <int PAIR, int BK>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, Params p) {
+    using C = Cfg<PAIR, BK>;
+    constexpr int NKB = C::NKB;
+    constexpr int A_BYTES = C::A_BYTES;
+    constexpr int SFA_BYTES = C::SFA_BYTES;
+    constexpr int SFB_BYTES = C::SFB_BYTES;
+    constexpr uint32_t SF_COLS_PER_STAGE = C::SF_COLS_PER_STAGE;
+    constexpr uint32_t SFB_OFF = C::SFB_OFF;
+    static_assert(sizeof(Smem) <= BARRIER_BYTES, "barrier area");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Smem* s = reinterpret_cast<Smem*>(base + STAGES * STAGE_BYTES);
-    auto stage_a = [&](int st) { return base + st * STAGE_BYTES; };
-    auto stage_b = [&](int st) { return base + st * STAGE_BYTES + A_BYTES; };
-    auto stage_sfa = [&](int st) { return base + st * STAGE_BYTES + A_BYTES + B_BYTES; };
-    auto stage_sfb = [&](int st) { return base + st * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; };
+    Smem* s = reinterpret_cast<Smem*>(base + C::STAGES * C::STAGE_BYTES);
+    auto stage_a = [&](int st) { return base + st * C::STAGE_BYTES; };
+    auto stage_b = [&](int st) { return base + st * C::STAGE_BYTES + A_BYTES; };
+    auto stage_sfa = [&](int st) { return base + st * C::STAGE_BYTES + A_BYTES + C::B_BYTES; };
+    auto stage_sfb = [&](int st) { return base + st * C::STAGE_BYTES + A_BYTES + C::B_BYTES + SFA_BYTES; };
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0;     // 0: the CTA that issues MMAs
+    const int unit = blockIdx.x / PAIR;                         // tile-processing unit (CTA or pair)
+    const int units = gridDim.x / PAIR;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&s->full[i], 1);
-            mbar_init(&s->sf_ready[i], SF_WARPS);
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(&s->ready[i], 1 + SF_WARPS * PAIR);   // producer of CTA 0 + scale writers
+            mbar_init(&s->sf_full[i], 1);
             mbar_init(&s->empty[i], 1);
         }
         mbar_init(&s->acc_full, 1);
-        mbar_init(&s->acc_empty, EPI_WARPS);
+        mbar_init(&s->acc_empty, EPI_WARPS * PAIR);
         mbar_init(&s->drain, 1);
         s->abort_flag = 0;
         fence_mbar_init();
@@ -135,11 +197,17 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         prefetch_tmap(&tmap_b);
     }
     if (warp == 1) {
-        tmem_alloc(&s->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR == 2) {
+            tmem_alloc_pair(&s->tmem_base, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&s->tmem_base, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR == 2) cluster_sync();      // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem = s->tmem_base;
     const volatile int* abort_flag = &s->abort_flag;
@@ -152,9 +220,13 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             uint32_t pending = 0;           // stages with a load in flight
             uint32_t pending_phase = 0;     // parity of that load's phase
             bool skip = p.fault_skip_first_load != 0;
-            for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
+            for (int tile = unit; tile < p.tiles && !*abort_flag; tile += units) {
                 int mb, nb;
                 tile_coords(tile, p, mb, nb);
+                const int arow = mb * C::TILE_M + (int)rank * BM;          // this CTA's A rows
+                const int brow = nb * BN + (int)rank * C::B_ROWS;          // this CTA's B rows
+                // scale rows past the padded end feed only discarded outputs
+                const int64_t at = min(arow / 128, p.a_row_tiles - 1);
                 for (int kt = 0; kt < p.k_stages; ++kt) {
                     if (!mbar_wait_bounded(&s->empty[st], phase ^ 1, p.timeout, abort_flag)) {
                         raise_abort(s, p);
@@ -162,40 +234,52 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     }
                     pending &= ~(1u << st);
                     const int nkb = min(NKB, p.kblocks - kt * NKB);
-                    const uint32_t sf_a = nkb * 512;
-                    if (skip) {     // test hook: never complete this stage
+                    const uint32_t sf_bytes = nkb * 512;               // one 128-row scale slice
+                    if (skip) {     // failure-detection test hook: never complete this stage
                         skip = false;
                     } else {
-                        mbar_arrive_expect_tx(&s->full[st], A_BYTES + B_BYTES + 3 * sf_a);
-                        tma_load_2d(stage_a(st), &tmap_a, &s->full[st], kt * (BK / 2), mb * BM);
-                        tma_load_2d(stage_b(st), &tmap_b, &s->full[st], kt * (BK / 2), nb * BN);
-                        const int64_t ka = (int64_t)kt * NKB;   // first k-atom of the stage
-                        bulk_load(stage_sfa(st), p.a_scales + ((int64_t)mb * p.katoms + ka) * 512, sf_a, &s->full[st]);
+                        // block scales first: small, and the scale writers start on them
+                        mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
+                        const int64_t ka = (int64_t)kt * NKB;              // first k-atom of the stage
+                        bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
                         for (int rt = 0; rt < 2; ++rt) {
-                            // rows past the padded end of B feed only discarded columns
                             const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
                             bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
-                                      p.b_scales + (bt * p.katoms + ka) * 512, sf_a, &s->full[st]);
+                                      p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                        }
+                        if (PAIR == 2) {
+                            // both CTAs' code tiles complete on CTA 0's barrier
+                            if (rank == 0) mbar_arrive_expect_tx(&s->ready[st], 2 * (A_BYTES + C::B_BYTES));
+                            const uint32_t bar0 = mapa_shared(smem_u32(&s->ready[st]), 0);
+                            tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
+                            tma_load_2d_pair(stage_b(st), &tmap_b, bar0, kt * C::ROW_BYTES, brow);
+                        } else {
+                            mbar_arrive_expect_tx(&s->ready[st], A_BYTES + C::B_BYTES);
+                            tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
+                            tma_load_2d(stage_b(st), &tmap_b, &s->ready[st], kt * C::ROW_BYTES, brow);
                         }
                         pending |= 1u << st;
                         pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
                     }
-                    if (++st == STAGES) { st = 0; phase ^= 1; }
+                    if (++st == C::STAGES) { st = 0; phase ^= 1; }
                 }
             }
             if (*abort_flag) {
                 // let the copies this thread issued land before the CTA exits
-                for (int i = 0; i < STAGES; ++i)
-                    if (pending & (1u << i))
-                        mbar_wait_bounded(&s->full[i], (pending_phase >> i) & 1, p.timeout, nullptr);
+                for (int i = 0; i < C::STAGES; ++i)
+                    if (pending & (1u << i)) {
+                        mbar_wait_bounded(&s->sf_full[i], (pending_phase >> i) & 1, p.timeout, nullptr);
+                        if (rank == 0)
+                            mbar_wait_bounded(&s->ready[i], (pending_phase >> i) & 1, p.timeout, nullptr);
+                    }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             int st = 0;
             uint32_t phase = 0, acc_phase = 0;
-            for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
+            for (int tile = unit; tile < p.tiles && !*abort_flag; tile += units) {
                 if (!mbar_wait_bounded(&s->acc_empty, acc_phase ^ 1, p.timeout, abort_flag)) {
                     raise_abort(s, p);
                     break;
@@ -203,8 +287,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < p.k_stages; ++kt) {
-                    // the stage's data is in shared memory and its scales in TMEM
-                    if (!mbar_wait_bounded(&s->sf_ready[st], phase, p.timeout, abort_flag)) {
+                    // the stage's codes are in shared memory and its scales in TMEM
+                    if (!mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag)) {
                         raise_abort(s, p);
                         ok = false;
                         break;
@@ -214,20 +298,25 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     const uint32_t a0 = smem_u32(stage_a(st)), b0 = smem_u32(stage_b(st));
                     const uint32_t sf = tmem + SF_COL + st * SF_COLS_PER_STAGE;
                     for (int kb = 0; kb < nkb; ++kb) {
-                        const uint64_t ad = smem_desc(a0 + kb * (MMA_K / 2), 16, 1024, 2);
-                        const uint64_t bd = smem_desc(b0 + kb * (MMA_K / 2), 16, 1024, 2);
-                        mma_mxf4nvf4(tmem + ACC_COL, ad, bd, IDESC, sf + kb * 4, sf + SFB_OFF + kb * 8,
-                                     (kt | kb) != 0);
+                        const uint64_t ad = smem_desc(a0 + kb * (MMA_K / 2), 16, C::SBO, C::SWIZZLE);
+                        const uint64_t bd = smem_desc(b0 + kb * (MMA_K / 2), 16, C::SBO, C::SWIZZLE);
+                        if (PAIR == 2)
+                            mma_mxf4nvf4_pair(tmem + ACC_COL, ad, bd, C::IDESC, sf + kb * 4, sf + SFB_OFF + kb * 8,
+                                              (kt | kb) != 0);
+                        else
+                            mma_mxf4nvf4(tmem + ACC_COL, ad, bd, C::IDESC, sf + kb * 4, sf + SFB_OFF + kb * 8,
+                                         (kt | kb) != 0);
                     }
-                    mma_commit(&s->empty[st]);
-                    if (++st == STAGES) { st = 0; phase ^= 1; }
+                    commit_to_all<PAIR>(&s->empty[st]);
+                    if (++st == C::STAGES) { st = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                mma_commit(&s->acc_full);
+                commit_to_all<PAIR>(&s->acc_full);
                 acc_phase ^= 1;
             }
             // no MMA may still be running when TMEM is released
-            mma_commit(&s->drain);
+            if (PAIR == 2) mma_commit_pair_mc(&s->drain, 0x1);
+            else mma_commit(&s->drain);
             mbar_wait_bounded(&s->drain, 0, p.timeout, nullptr);
         }
     } else if (warp < FIRST_EPI_WARP) {
@@ -238,10 +327,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         const int quad = warp & 3;
         int st = 0;
         uint32_t phase = 0;
-        for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
+        for (int tile = unit; tile < p.tiles; tile += units) {
             bool ok = true;
             for (int kt = 0; kt < p.k_stages; ++kt) {
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s->full[st], phase, p.timeout, abort_flag));
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s->sf_full[st], phase, p.timeout, abort_flag));
                 if (!ok) break;
                 const int nkb = min(NKB, p.kblocks - kt * NKB);
                 const uint8_t* sfa = stage_sfa(st) + lane * 16;
@@ -256,8 +345,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s->sf_ready[st]);
-                if (++st == STAGES) { st = 0; phase ^= 1; }
+                if (lane == 0) arrive_leader<PAIR>(&s->ready[st]);
+                if (++st == C::STAGES) { st = 0; phase ^= 1; }
             }
             if (!ok) {
                 if (lane == 0) raise_abort(s, p);
@@ -271,7 +360,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         const float ab = __fmul_rn(__ldg(p.alpha_a), __ldg(p.alpha_b));
         const bool vec_ok = (p.N % 8) == 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
+        for (int tile = unit; tile < p.tiles; tile += units) {
             // warp-uniform decisions: tcgen05.ld below is .sync.aligned
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             int mb, nb;
@@ -282,7 +371,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 break;
             }
             tc_fence_after();
-            const int row = mb * BM + quad * 32 + lane;
+            const int row = mb * C::TILE_M + (int)rank * BM + quad * 32 + lane;
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
             const int colh = nb * BN + half * 128;
             if (vec_ok && nb * BN + BN <= p.N) {
@@ -302,7 +391,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s->acc_empty);
+                if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
                 if (row < p.M) {
                     uint4* d4 = reinterpret_cast<uint4*>(p.y + (int64_t)row * p.N + colh);
 #pragma unroll
@@ -314,7 +403,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 }
             } else {
                 // Ragged right edge (or N not a multiple of 8): one 32-column
-                // chunk at a time, element stores past the last full chunk.
+                // chunk at a time, element stores.
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(taddr + c * 32, r);
@@ -322,7 +411,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     if (c == 3) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&s->acc_empty);
+                        if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
                     }
                     const int col0 = colh + c * 32;
                     if (row >= p.M || col0 >= p.N) continue;
@@ -343,9 +432,11 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
     __syncwarp();   // reconverge the single-lane roles before the block barrier
     tc_fence_before();
     __syncthreads();
+    if (PAIR == 2) cluster_sync();      // the peer's MMAs and arrivals are finished
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        if (PAIR == 2) tmem_dealloc_pair(tmem, TMEM_COLS);
+        else tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -368,31 +459,64 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D byte tensor [rows, K/2] with a box of `box_rows` x 128 bytes, 128-byte swizzle.
-static bool make_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+// 2-D byte tensor [rows, K/2] with a box of `box_rows` rows x `box_bytes`
+// bytes (128 or 64) in the matching 128- or 64-byte swizzle.
+static bool make_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows,
+                          int box_bytes) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)(gemm::BK / 2), (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+namespace {
+
+struct FormState {
+    bool attr_set = false;
+    int max_units = 0;      // co-resident CTAs (PAIR 1) or clusters (PAIR 2)
+};
+FormState g_form[64][3][2];
+
+template <int PAIR, int BK>
+cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     using namespace gemm;
-    static bool attr_set[64] = {};
+    using C = Cfg<PAIR, BK>;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][BK == 256];
+    if (!fs.attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm<PAIR, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        fs.max_units = num_sms / PAIR;
+        if (PAIR == 2) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(2 * fs.max_units);
+            cfg.blockDim = dim3(THREADS);
+            cfg.dynamicSmemBytes = C::SMEM_BYTES;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, k_gemm<PAIR, BK>, &cfg) == cudaSuccess && clusters > 0)
+                fs.max_units = std::min(fs.max_units, clusters);
+            cudaGetLastError();
+        }
+        fs.attr_set = true;
     }
     CUtensorMap ma, mb;
-    if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM) || !make_code_map(&mb, a.b_codes, a.N, a.K, BN))
+    if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM, C::ROW_BYTES) ||
+        !make_code_map(&mb, a.b_codes, a.N, a.K, C::B_ROWS, C::ROW_BYTES))
         return cudaErrorInvalidValue;
     Params p{};
     p.a_scales = a.a_scales;
@@ -403,19 +527,55 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.M = (int)a.M;
     p.N = (int)a.N;
     p.K = (int)a.K;
-    p.m_blocks = (int)((a.M + BM - 1) / BM);
+    p.m_blocks = (int)((a.M + C::TILE_M - 1) / C::TILE_M);
     p.n_blocks = (int)((a.N + BN - 1) / BN);
     p.tiles = p.m_blocks * p.n_blocks;
     p.kblocks = (int)(a.K / MMA_K);
-    p.k_stages = (p.kblocks + NKB - 1) / NKB;
+    p.k_stages = (p.kblocks + C::NKB - 1) / C::NKB;
     p.katoms = (int)scale_atom_cols(a.K);
+    p.a_row_tiles = (int)(padded_rows(a.M) / 128);
     p.b_row_tiles = (int)(padded_rows(a.N) / 128);
     p.status = a.status;
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
-    const int grid = std::min(p.tiles, num_sms);
-    k_gemm<<<grid, THREADS, SMEM_BYTES, stream>>>(ma, mb, p);
-    return cudaGetLastError();
+    const int units = std::min(p.tiles, fs.max_units);
+    if (PAIR == 1) {
+        k_gemm<1, BK><<<units, THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * units);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_gemm<PAIR, BK>, ma, mb, p);
+}
+
+int env_choice(const char* name, int a, int b, int dflt) {
+    const char* v = getenv(name);
+    if (!v) return dflt;
+    const int x = atoi(v);
+    return (x == a || x == b) ? x : dflt;
+}
+
+}  // namespace
+
+// The 2-CTA form for M > 128, the 1-CTA form otherwise.  MQ_GEMM_FORM=1|2 and
+// MQ_GEMM_BK=128|256 force a variant (the tests check every variant on the
+// same shapes).
+cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+    const int form = env_choice("MQ_GEMM_FORM", 1, 2, a.M > gemm::BM ? 2 : 1);
+    const int bk = env_choice("MQ_GEMM_BK", 128, 256, 256);
+    if (form == 2)
+        return bk == 128 ? launch_form<2, 128>(a, num_sms, stream) : launch_form<2, 256>(a, num_sms, stream);
+    return bk == 128 ? launch_form<1, 128>(a, num_sms, stream) : launch_form<1, 256>(a, num_sms, stream);
 }
 
 }  // namespace mq

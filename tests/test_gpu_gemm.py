@@ -18,6 +18,18 @@ pytestmark = pytest.mark.gpu
 TOL = 1e-3
 
 
+@pytest.fixture(params=["auto", "1-128", "1-256", "2-128", "2-256"])
+def gemm_form(request, monkeypatch):
+    """Run a test with the library's choice of GEMM variant, then forced to
+    each of: one CTA (128 x 256 tiles) or a CTA pair (256 x 256 tiles), with
+    128 or 256 K elements per pipeline stage."""
+    if request.param != "auto":
+        form, bk = request.param.split("-")
+        monkeypatch.setenv("MQ_GEMM_FORM", form)
+        monkeypatch.setenv("MQ_GEMM_BK", bk)
+    return request.param
+
+
 def _gemm(qa, qb, M, N, K):
     y = torch.empty(M, N, dtype=torch.bfloat16, device=dev())
     ws = mq.workspace(mq.mq_workspace_bytes(), dev())
@@ -36,8 +48,9 @@ def _upload(codes_np, logical_scales, K, alpha):
     return q
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (128, 256, 256), (200, 300, 512), (1, 8, 64), (257, 513, 320)])
-def test_exact_products_bit_exact(M, N, K):
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (128, 256, 256), (200, 300, 512), (1, 8, 64), (257, 513, 320),
+                                   (512, 512, 256)])
+def test_exact_products_bit_exact(M, N, K, gemm_form):
     """Codes random, scales powers of two in [2^-2, 2^2], alpha = 1: every
     partial sum is exact in binary32, so Y must equal the oracle bit for bit.
     Pins the MMA's reading of code nibbles, E4M3 scales and the scale order."""
@@ -78,7 +91,7 @@ def _random_case(M, N, K, seed, student_t=False):
 
 @pytest.mark.parametrize("M,N,K", [(128, 1024, 1024), (1, 256, 64), (3, 17, 128), (17, 3, 64), (130, 300, 320),
                                    (257, 513, 1024), (300, 257, 128), (512, 1024, 4096), (96, 4096, 12288)])
-def test_gemm_random_against_oracle(M, N, K):
+def test_gemm_random_against_oracle(M, N, K, gemm_form):
     x, w = _random_case(M, N, K, seed=M + N + K)
     ax, xc, xs, qx = gpu_quantize(x)
     aw, wc, wsc, qw = gpu_quantize(w)
