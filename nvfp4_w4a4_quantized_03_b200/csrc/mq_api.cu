@@ -1,6 +1,7 @@
 // mq_api.cu -- the extern "C" boundary of libmq.so (declared in include/mq.h):
 // argument validation, per-device attribute cache, and the launches.
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -48,6 +49,8 @@ size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 int check_rows_k(int64_t rows, int64_t K) {
     if (rows <= 0 || K <= 0 || K % 64 != 0) return MQ_ERR_SHAPE;
     if (rows > (int64_t)1 << 31 || K > (int64_t)1 << 24) return MQ_ERR_SHAPE;
+    // the quantizers index 16-element blocks of the (row-padded) tensor in 32 bits
+    if ((rows + 127) / 128 * 128 * (K / 16) >= ((int64_t)1 << 31)) return MQ_ERR_SHAPE;
     return MQ_OK;
 }
 
@@ -83,9 +86,14 @@ size_t mq_nvfp4_scales_bytes(int64_t rows, int64_t K) {
 
 size_t mq_workspace_bytes(void) { return mq::WS_HEADER_BYTES; }
 
+// Workspace of mq_linear_w4a4: header | readiness flags of the fused kernel |
+// codes of X | scales of X.
+static size_t linear_flags_bytes(int64_t M, int64_t K) { return round256((size_t)mq::fused_flag_count(M, K) * 4); }
+
 size_t mq_linear_w4a4_workspace_bytes(int64_t M, int64_t K) {
     if (M <= 0 || K <= 0) return 0;
-    return mq::WS_HEADER_BYTES + round256(mq_nvfp4_codes_bytes(M, K)) + round256(mq_nvfp4_scales_bytes(M, K));
+    return mq::WS_HEADER_BYTES + linear_flags_bytes(M, K) + round256(mq_nvfp4_codes_bytes(M, K)) +
+           round256(mq_nvfp4_scales_bytes(M, K));
 }
 
 int mq_tensor_scale(const void* x, int64_t numel, float* alpha, void* ws, size_t ws_bytes, void* stream) {
@@ -160,13 +168,33 @@ int mq_linear_w4a4(const void* x, int64_t M, int64_t K, const uint8_t* w_codes, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t* words = static_cast<uint32_t*>(ws);
     float* alpha_x = reinterpret_cast<float*>(words + mq::WS_ALPHA);
-    uint8_t* x_codes = static_cast<uint8_t*>(ws) + mq::WS_HEADER_BYTES;
+    int* flags = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + mq::WS_HEADER_BYTES);
+    uint8_t* x_codes = reinterpret_cast<uint8_t*>(flags) + linear_flags_bytes(M, K);
     uint8_t* x_scales = x_codes + round256(mq_nvfp4_codes_bytes(M, K));
-    cudaError_t e = mq::launch_amax(x, M * K, words, alpha_x, sms, s);
-    if (e == cudaSuccess) e = mq::launch_quantize(x, M, K, alpha_x, x_codes, x_scales, s);
-    if (e != cudaSuccess) return MQ_ERR_CUDA;
     mq::GemmArgs g{x_codes, x_scales, alpha_x, w_codes, w_scales, alpha_w, y, M, N, K,
                    reinterpret_cast<int*>(words + mq::WS_STATUS), DEFAULT_TIMEOUT_CYCLES, 0};
+    // MQ_LINEAR_PATH selects how X is quantized (all three give identical Y):
+    //   "onepass" (default) one cooperative kernel: amax, grid barrier,
+    //                       quantization of the data the amax pass left in L2;
+    //   "split"             mq_tensor_scale's and mq_nvfp4_quantize's kernels;
+    //   "ingemm"            amax kernel, then quantizer warps inside the GEMM.
+    const char* path = getenv("MQ_LINEAR_PATH");
+    const char mode = path ? path[0] : 'o';
+    cudaError_t e = cudaSuccess;
+    if (mode == 'i') {
+        // amax (which also clears the readiness flags), then the GEMM with
+        // the activation's quantization done by its quantizer warps
+        e = mq::launch_amax(x, M * K, words, alpha_x, sms, s, flags, (int)mq::fused_flag_count(M, K));
+        g.x = x;
+        g.flags = flags;
+    } else if (mode == 's') {
+        e = mq::launch_amax(x, M * K, words, alpha_x, sms, s);
+        if (e == cudaSuccess) e = mq::launch_quantize(x, M, K, alpha_x, x_codes, x_scales, s);
+    } else {
+        e = mq::launch_quantize_onepass(x, M, K, words, alpha_x, x_codes, x_scales,
+                                        reinterpret_cast<int*>(words + mq::WS_STATUS), DEFAULT_TIMEOUT_CYCLES, s);
+    }
+    if (e != cudaSuccess) return MQ_ERR_CUDA;
     return cuda_status(mq::launch_gemm(g, sms, s));
 }
 

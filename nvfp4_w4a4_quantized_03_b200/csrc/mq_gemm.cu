@@ -24,7 +24,14 @@
 //   warp 1      allocates TMEM; in the (even) CTA one lane issues
 //               tcgen05.mma (K = 64 per instruction, 4 per stage) and
 //               tcgen05.commit to release stages and to publish a tile.
-//   warps 2..5  scale writers: move each stage's block scales from shared
+//   warps 2..3  fused linear only (QUANT): quantizer warps.  They quantize the
+//               bf16 activation X into A's codes and scales (mq_nvfp4.cuh),
+//               32 rows x one K stage at a time, in the order the tile raster
+//               consumes them, and publish each 128-row x stage block with a
+//               release-add on a global flag; the producer acquires the flag
+//               before loading that block, so X is quantized once, inside the
+//               GEMM, with HBM bandwidth the GEMM leaves idle.
+//   warps 4..7  scale writers: move each stage's block scales from shared
 //               memory into that stage's TMEM scale columns with tcgen05.st
 //               and arrive on CTA 0's `ready` barrier (one barrier per stage
 //               is all the MMA thread waits on),
@@ -33,7 +40,7 @@
 //               costs the tensor pipe nothing, where tcgen05.cp issued by the
 //               MMA thread measured ~45 cycles per copy, serialised with the
 //               MMAs.
-//   warps 6..13 epilogue: drain the CTA's 128 x 256 fp32 accumulator into
+//   warps 8..15 epilogue: drain the CTA's 128 x 256 fp32 accumulator into
 //               registers (scaled by alpha_a * alpha_b, rounded to bf16),
 //               release it to the MMA thread, then store.
 // Every wait on an mbarrier is bounded; on a timeout the kernel records
@@ -45,6 +52,7 @@
 #include <cstdlib>
 
 #include "mq_internal.h"
+#include "mq_nvfp4.cuh"
 #include "mq_ptx.cuh"
 
 namespace mq {
@@ -53,9 +61,11 @@ namespace gemm {
 constexpr int BM = 128;               // A rows per CTA (TMEM lanes)
 constexpr int BN = 256;               // accumulator columns (N of one MMA)
 constexpr int MMA_K = 64;             // K elements per tcgen05.mma (kind::mxf4nvf4)
+constexpr int QUANT_WARPS = 2;
 constexpr int SF_WARPS = 4;
 constexpr int EPI_WARPS = 8;
-constexpr int FIRST_SF_WARP = 2;
+constexpr int FIRST_Q_WARP = 2;
+constexpr int FIRST_SF_WARP = FIRST_Q_WARP + QUANT_WARPS;     // a warpgroup: one warp per TMEM sub-partition
 constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + SF_WARPS;
 constexpr int THREADS = (FIRST_EPI_WARP + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
@@ -113,6 +123,10 @@ struct Params {
     int* status;
     long long timeout;
     int fault_skip_first_load;
+    const uint16_t* x;       // fused linear: bf16 activation [M, K]
+    uint8_t* x_codes;        // fused linear: where A's codes are written
+    uint8_t* x_scales;       // fused linear: where A's scales are written
+    int* flags;              // fused linear: [a_row_tiles][k_stages] slab counts
 };
 
 struct Smem {
@@ -155,7 +169,7 @@ __device__ __forceinline__ void commit_to_all(uint64_t* bar) {
     else mma_commit(bar);
 }
 
-template <int PAIR, int BK>
+template <int PAIR, int BK, bool QUANT>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, Params p) {
     using C = Cfg<PAIR, BK>;
@@ -238,26 +252,38 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     if (skip) {     // failure-detection test hook: never complete this stage
                         skip = false;
                     } else {
-                        // block scales first: small, and the scale writers start on them
-                        mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
                         const int64_t ka = (int64_t)kt * NKB;              // first k-atom of the stage
-                        bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                        // B's block scales and codes first: they never wait
+                        mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
                         for (int rt = 0; rt < 2; ++rt) {
                             const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
                             bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
                                       p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
                         }
+                        uint32_t bar0 = 0;
                         if (PAIR == 2) {
                             // both CTAs' code tiles complete on CTA 0's barrier
                             if (rank == 0) mbar_arrive_expect_tx(&s->ready[st], 2 * (A_BYTES + C::B_BYTES));
-                            const uint32_t bar0 = mapa_shared(smem_u32(&s->ready[st]), 0);
-                            tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
+                            bar0 = mapa_shared(smem_u32(&s->ready[st]), 0);
                             tma_load_2d_pair(stage_b(st), &tmap_b, bar0, kt * C::ROW_BYTES, brow);
                         } else {
                             mbar_arrive_expect_tx(&s->ready[st], A_BYTES + C::B_BYTES);
-                            tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
                             tma_load_2d(stage_b(st), &tmap_b, &s->ready[st], kt * C::ROW_BYTES, brow);
                         }
+                        if (QUANT && arow / 128 < p.a_row_tiles) {
+                            // A's block (arow, kt) is written by quantizer warps (of any CTA)
+                            const int* f = p.flags + (int64_t)(arow / 128) * p.k_stages + kt;
+                            if (ld_acquire_gpu(f) < 4) {
+                                const long long t0 = clock64();
+                                while (ld_acquire_gpu(f) < 4) {
+                                    if (*abort_flag || clock64() - t0 > p.timeout) { raise_abort(s, p); break; }
+                                }
+                            }
+                            fence_proxy_async_global();
+                        }
+                        bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                        if (PAIR == 2) tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
+                        else tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
                         pending |= 1u << st;
                         pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
                     }
@@ -318,6 +344,71 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             if (PAIR == 2) mma_commit_pair_mc(&s->drain, 0x1);
             else mma_commit(&s->drain);
             mbar_wait_bounded(&s->drain, 0, p.timeout, nullptr);
+        }
+    } else if (warp < FIRST_SF_WARP) {
+        // ------------------------------------------------------------ quantizer warps (fused linear)
+        if constexpr (QUANT) {
+            // A unit is 32 rows x one K stage (BK elements, BK / 16 blocks per
+            // row).  Units are numbered in the order the tile raster consumes
+            // them: raster group of GROUP_M tile rows, then K stage, then
+            // 32-row slab; unit u goes to quantizer warp u mod (all warps).
+            static_assert(BK == 256, "the fused quantizer maps one lane to each of a row's 16 blocks");
+            const int qw = blockIdx.x * QUANT_WARPS + (warp - FIRST_Q_WARP);
+            const int nqw = gridDim.x * QUANT_WARPS;
+            const int slabs = p.a_row_tiles * 4;
+            const int slabs_per_group = GROUP_M * C::TILE_M / 32;
+            const int64_t per_group = (int64_t)slabs_per_group * p.k_stages;
+            const int64_t units = (int64_t)slabs * p.k_stages;
+            const float alpha = *p.alpha_a;
+            const int nblk = p.K / 16;
+            const int half = lane >> 4;             // which of the two rows of an iteration
+            const int kbl = lane & 15;              // block column within the stage
+            for (int64_t u = qw; u < units; u += nqw) {
+                if (*abort_flag) break;
+                const int g = (int)(u / per_group);
+                const int first = g * slabs_per_group;
+                const int ns = min(slabs_per_group, slabs - first);
+                const int64_t ul = u - (int64_t)g * per_group;
+                const int kt = (int)(ul / ns);
+                const int slab = first + (int)(ul % ns);
+                const int kb = kt * (BK / 16) + kbl;
+                const bool col_ok = kb < nblk;
+#pragma unroll 1
+                for (int batch = 0; batch < 2; ++batch) {
+                    uint4 v[8][2];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int row = slab * 32 + (batch * 8 + j) * 2 + half;
+                        if (row < p.M && col_ok) {
+                            const uint4* src = reinterpret_cast<const uint4*>(p.x + (int64_t)row * p.K + kb * 16);
+                            v[j][0] = src[0];
+                            v[j][1] = src[1];
+                        } else {
+                            v[j][0] = make_uint4(0, 0, 0, 0);
+                            v[j][1] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int row = slab * 32 + (batch * 8 + j) * 2 + half;
+                        uint32_t c0 = 0, c1 = 0, sc = 0;
+                        if (row < p.M && col_ok) {
+                            sc = quantize_block16(v[j][0], v[j][1], alpha, c0, c1);
+                            *reinterpret_cast<uint2*>(p.x_codes + (int64_t)row * (p.K / 2) + kb * 8) =
+                                make_uint2(c0, c1);
+                        }
+                        // four consecutive block columns form one 32-bit scale word
+                        uint32_t word = sc << (8 * (kbl & 3));
+                        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+                        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+                        if ((kbl & 3) == 0 && col_ok)
+                            *reinterpret_cast<uint32_t*>(p.x_scales + scale_byte_offset(row, kb, p.katoms)) = word;
+                    }
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) red_release_gpu_add(p.flags + (int64_t)(slab / 4) * p.k_stages + kt, 1);
+            }
         }
     } else if (warp < FIRST_EPI_WARP) {
         // ------------------------------------------------------------ scale writers
@@ -481,18 +572,18 @@ struct FormState {
     bool attr_set = false;
     int max_units = 0;      // co-resident CTAs (PAIR 1) or clusters (PAIR 2)
 };
-FormState g_form[64][3][2];
+FormState g_form[64][3][2][2];
 
-template <int PAIR, int BK>
+template <int PAIR, int BK, bool QUANT>
 cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     using namespace gemm;
     using C = Cfg<PAIR, BK>;
     int dev = 0;
     cudaGetDevice(&dev);
-    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][BK == 256];
+    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][BK == 256][QUANT];
+    auto kernel = k_gemm<PAIR, BK, QUANT>;
     if (!fs.attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm<PAIR, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         fs.max_units = num_sms / PAIR;
         if (PAIR == 2) {
@@ -508,7 +599,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int clusters = 0;
-            if (cudaOccupancyMaxActiveClusters(&clusters, k_gemm<PAIR, BK>, &cfg) == cudaSuccess && clusters > 0)
+            if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) == cudaSuccess && clusters > 0)
                 fs.max_units = std::min(fs.max_units, clusters);
             cudaGetLastError();
         }
@@ -538,24 +629,35 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.status = a.status;
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
+    p.x = static_cast<const uint16_t*>(a.x);
+    p.x_codes = const_cast<uint8_t*>(a.a_codes);
+    p.x_scales = const_cast<uint8_t*>(a.a_scales);
+    p.flags = a.flags;
     const int units = std::min(p.tiles, fs.max_units);
-    if (PAIR == 1) {
-        k_gemm<1, BK><<<units, THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
-        return cudaGetLastError();
-    }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * units);
+    cudaLaunchAttribute attr[2];
+    int nattr = 0;
+    if (PAIR == 2) {
+        attr[nattr].id = cudaLaunchAttributeClusterDimension;
+        attr[nattr].val.clusterDim.x = 2;
+        attr[nattr].val.clusterDim.y = 1;
+        attr[nattr].val.clusterDim.z = 1;
+        ++nattr;
+    }
+    if (QUANT) {
+        // producers wait on quantizer warps of other CTAs: every CTA must be
+        // resident at once, which a cooperative launch guarantees (or refuses)
+        attr[nattr].id = cudaLaunchAttributeCooperative;
+        attr[nattr].val.cooperative = 1;
+        ++nattr;
+    }
+    cfg.gridDim = dim3(PAIR * units);
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_gemm<PAIR, BK>, ma, mb, p);
+    cfg.numAttrs = nattr;
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
 }
 
 int env_choice(const char* name, int a, int b, int dflt) {
@@ -567,15 +669,24 @@ int env_choice(const char* name, int a, int b, int dflt) {
 
 }  // namespace
 
+int64_t fused_flag_count(int64_t M, int64_t K) {
+    using C = gemm::Cfg<2, 256>;
+    return padded_rows(M) / 128 * ((K / gemm::MMA_K + C::NKB - 1) / C::NKB);
+}
+
 // The 2-CTA form for M > 128, the 1-CTA form otherwise.  MQ_GEMM_FORM=1|2 and
 // MQ_GEMM_BK=128|256 force a variant (the tests check every variant on the
-// same shapes).
+// same shapes); the fused linear always runs with 256-element K stages.
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     const int form = env_choice("MQ_GEMM_FORM", 1, 2, a.M > gemm::BM ? 2 : 1);
+    if (a.x) return form == 2 ? launch_form<2, 256, true>(a, num_sms, stream)
+                              : launch_form<1, 256, true>(a, num_sms, stream);
     const int bk = env_choice("MQ_GEMM_BK", 128, 256, 256);
     if (form == 2)
-        return bk == 128 ? launch_form<2, 128>(a, num_sms, stream) : launch_form<2, 256>(a, num_sms, stream);
-    return bk == 128 ? launch_form<1, 128>(a, num_sms, stream) : launch_form<1, 256>(a, num_sms, stream);
+        return bk == 128 ? launch_form<2, 128, false>(a, num_sms, stream)
+                         : launch_form<2, 256, false>(a, num_sms, stream);
+    return bk == 128 ? launch_form<1, 128, false>(a, num_sms, stream)
+                     : launch_form<1, 256, false>(a, num_sms, stream);
 }
 
 }  // namespace mq

@@ -14,6 +14,7 @@ enum WsWord : int {
     WS_TICKET = 1,      // blocks of the amax pass that have finished
     WS_STATUS = 2,      // device-side status (0 = ok, else an mq_status code)
     WS_ALPHA = 3,       // alpha_x written by the amax pass of mq_linear_w4a4
+    WS_GENERATION = 4,  // grid-barrier generation of the one-pass quantizer (only grows)
 };
 constexpr size_t WS_HEADER_BYTES = 256;
 
@@ -24,9 +25,14 @@ __host__ __device__ inline int64_t padded_rows(int64_t rows) { return (rows + 12
 
 // Launchers (enqueue on `stream`, no synchronisation).
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
-                        int num_sms, cudaStream_t stream);
+                        int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0);
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+// alpha_x and the NVFP4 codes/scales of x in one cooperative launch (amax
+// pass, grid barrier, quantization pass over recently read data).
+cudaError_t launch_quantize_onepass(const void* x, int64_t rows, int64_t K, uint32_t* ws_words, float* alpha_out,
+                                    uint8_t* codes, uint8_t* scales, int* status, long long timeout_cycles,
+                                    cudaStream_t stream);
 
 struct GemmArgs {
     const uint8_t* a_codes;
@@ -40,7 +46,15 @@ struct GemmArgs {
     int* status;            // may be null
     long long timeout_cycles;
     int fault_skip_first_load;   // failure-detection tests only
+    // Fused activation quantization (mq_linear_w4a4): when x is set, the
+    // kernel's quantizer warps write A (a_codes / a_scales) from bf16 x with
+    // alpha_a, publishing each 128-row x (stage) block through `flags`.
+    const void* x = nullptr;
+    int* flags = nullptr;
 };
+
+// Readiness flags of the fused linear: one int per (128-row block, K stage).
+int64_t fused_flag_count(int64_t M, int64_t K);
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace mq

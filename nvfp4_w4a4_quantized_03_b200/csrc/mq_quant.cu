@@ -17,43 +17,34 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "mq_internal.h"
-#include "mq_ptx.cuh"
+#include "mq_nvfp4.cuh"
 
 namespace mq {
-
-// max over the two bf16 halves of |w|, kept packed: clearing the sign bits
-// leaves non-negative bf16 patterns, which order like unsigned integers.
-__device__ __forceinline__ uint32_t absmax2(uint32_t m, uint32_t w) {
-    return __vmaxu2(m, w & 0x7fff7fffu);
-}
-
-__device__ __forceinline__ uint32_t absmax_vec(uint32_t m, const uint4& v) {
-    m = absmax2(m, v.x);
-    m = absmax2(m, v.y);
-    m = absmax2(m, v.z);
-    return absmax2(m, v.w);
-}
 
 constexpr int AMAX_THREADS = 512;
 
 // One pass over x (16-byte vectors); every block folds its max into ws with
 // one atomic, and the last block to finish turns it into alpha and resets
-// the two counters to zero.
+// the two counters to zero.  `clear` (may be null) is zero-filled on the way:
+// the fused linear's readiness flags for this call.
 __global__ void __launch_bounds__(AMAX_THREADS)
 k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ tail, int ntail,
-       uint32_t* __restrict__ ws, float* __restrict__ alpha_out) {
+       uint32_t* __restrict__ ws, float* __restrict__ alpha_out, int* __restrict__ clear, int nclear) {
     uint32_t m = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; i + 3 * stride < nvec; i += 4 * stride) {
-        uint4 a = x[i], b = x[i + stride], c = x[i + 2 * stride], d = x[i + 3 * stride];
-        m = absmax_vec(m, a);
-        m = absmax_vec(m, b);
-        m = absmax_vec(m, c);
-        m = absmax_vec(m, d);
+    for (int64_t j = i; j < nclear; j += stride) clear[j] = 0;
+    // eight independent 16-byte loads in flight per thread on every pass
+    for (; i < nvec; i += 8 * stride) {
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = x[min(i + j * stride, nvec - 1)];   // a repeat leaves the max unchanged
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = absmax_vec(m, v[j]);
     }
-    for (; i < nvec; i += stride) m = absmax_vec(m, x[i]);
     if (blockIdx.x == 0 && (int)threadIdx.x < ntail) m = absmax2(m, tail[threadIdx.x]);
 
     uint32_t v = max(m & 0xffffu, m >> 16);
@@ -86,79 +77,181 @@ k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ t
 
 constexpr int QUANT_THREADS = 256;
 
-// Byte offset of (row, scale column kb) in the MMA scale layout: atoms of
-// 128 rows x 4 columns; inside an atom row r sits at (r % 32) * 16 +
-// ((r / 32) % 4) * 4 and column kb at kb % 4.
-__device__ __forceinline__ int64_t scale_byte_offset(int64_t row, int64_t kb, int64_t katoms) {
-    return ((row >> 7) * katoms + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3);
+// Quantizes the four consecutive 16-element blocks [4q, 4q + 4) of row `row`:
+// 128 bytes of x in, 32 code bytes and one 32-bit scale word (the four block
+// scales, one word of the MMA layout) out.  Padding rows (row >= rows) get a
+// zero scale word.
+__device__ __forceinline__ void quantize_quad(const uint4* __restrict__ x, int64_t rows, int64_t K, uint32_t row,
+                                              uint32_t q, float alpha, uint4* __restrict__ codes,
+                                              uint8_t* __restrict__ scales, const uint4 (&v)[8]) {
+    uint32_t word = 0;
+    if (row < rows) {
+        uint32_t c[8];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) word |= quantize_block16(v[2 * b], v[2 * b + 1], alpha, c[2 * b], c[2 * b + 1]) << (8 * b);
+        uint4* dst = codes + ((int64_t)row * (K / 64) + q) * 2;      // 32 bytes per quad
+        dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+        dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+    }
+    *reinterpret_cast<uint32_t*>(scales + scale_byte_offset(row, 4 * (int64_t)q, K / 64)) = word;
 }
 
-// One thread per 16-element block; threads run over the padded row range so
-// the padding rows of the scale buffer are written as zeros.
+__device__ __forceinline__ void load_quad(const uint4* __restrict__ x, int64_t rows, int64_t K, uint32_t row,
+                                          uint32_t q, uint4 (&v)[8]) {
+    if (row < rows) {
+        const uint4* src = x + ((int64_t)row * (K / 64) + q) * 8;      // 128 bytes per quad
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = src[j];
+    }
+}
+
+// One thread per four consecutive blocks of a row (K is a multiple of 64);
+// threads run over the padded row range so the padding rows of the scale
+// buffer are written as zeros.
 __global__ void __launch_bounds__(QUANT_THREADS)
 k_quantize(const uint4* __restrict__ x, int64_t rows, int64_t prows, int64_t K,
-           const float* __restrict__ alpha_p, uint2* __restrict__ codes,
-           uint8_t* __restrict__ scales) {
-    const int64_t nb = K >> 4;
+           const float* __restrict__ alpha_p, uint4* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const uint32_t quads = (uint32_t)(K / 64);
     const int64_t g = (int64_t)blockIdx.x * QUANT_THREADS + threadIdx.x;
-    const int64_t row = g / nb, kb = g - row * nb;
-    const bool in_pad = g < prows * nb;
-    const bool real = row < rows;
-    uint32_t sc = 0;
-    if (real) {
-        const uint4 v0 = x[2 * g], v1 = x[2 * g + 1];
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t m = absmax_vec(absmax_vec(0u, v0), v1);
-        const float amax_b = __uint_as_float(max(m & 0xffffu, m >> 16) << 16);
-        const float alpha = __ldg(alpha_p);
-        // sigma_b = Pi_E4M3(amax_b / (alpha * q_max))
-        const float t = __fdiv_rn(amax_b, __fmul_rn(6.0f, alpha));
-        sc = cvt_e4m3x2(0.0f, t) & 0xffu;
-        const float sigma = __half2float(__ushort_as_half((uint16_t)(cvt_e4m3x2_to_f16x2((uint16_t)sc) & 0xffffu)));
-        uint32_t c0 = 0, c1 = 0;
-        if (sigma != 0.0f) {
-            // q_i = Pi_E2M1(x_i / (alpha * sigma_b)), one reciprocal per block
-            const float r = __frcp_rn(__fmul_rn(alpha, sigma));
-            float f[16];
+    if (g >= prows * quads) return;
+    const uint32_t row = (uint32_t)g / quads, q = (uint32_t)g - row * quads;
+    uint4 v[8];
+    load_quad(x, rows, K, row, q, v);
+    quantize_quad(x, rows, K, row, q, __ldg(alpha_p), codes, scales, v);
+}
+
+constexpr int ONEPASS_THREADS = 256;
+
+// alpha_x and the codes/scales of a [rows, K] tensor in one launch.  Every
+// block is resident (cooperative launch).
+//   phase 1: max |x| over the whole tensor (eight 16-byte loads in flight per
+//            thread); blocks fold their max into ws with one atomic; the last
+//            block computes alpha_x, resets the counters and bumps the
+//            generation word, which releases all blocks (bounded spin).
+//   phase 2: one 16-element block per thread and step, walking the tensor
+//            from its end so the most recently read lines (still in L2) are
+//            quantized first.
+__global__ void __launch_bounds__(ONEPASS_THREADS, 4)
+k_quantize_onepass(const uint4* __restrict__ x, int64_t rows, int64_t prows, int64_t K,
+                   uint32_t* __restrict__ ws, float* __restrict__ alpha_out, uint4* __restrict__ codes,
+                   uint8_t* __restrict__ scales, int* __restrict__ status, long long timeout) {
+    __shared__ uint32_t red[ONEPASS_THREADS / 32];
+    __shared__ bool ok_shared;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(&ws[WS_GENERATION]);
+
+    // ---- phase 1: amax
+    const int64_t nvec = rows * K / 8;
+    const int64_t stride = (int64_t)gridDim.x * ONEPASS_THREADS;
+    int64_t i = (int64_t)blockIdx.x * ONEPASS_THREADS + threadIdx.x;
+    uint32_t m = 0;
+    for (; i < nvec; i += 8 * stride) {
+        uint4 v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                f[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), r);
-                f[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xffff0000u), r);
-            }
-            c0 = cvt_e2m1x8(f[0], f[1], f[2], f[3], f[4], f[5], f[6], f[7]);
-            c1 = cvt_e2m1x8(f[8], f[9], f[10], f[11], f[12], f[13], f[14], f[15]);
-        }
-        codes[g] = make_uint2(c0, c1);
+        for (int j = 0; j < 8; ++j) v[j] = x[min(i + j * stride, nvec - 1)];   // a repeat leaves the max unchanged
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = absmax_vec(m, v[j]);
     }
-    // Four consecutive scale columns of one row form one 32-bit word of the
-    // layout; lanes 4j..4j+3 hold them (nb is a multiple of 4).
-    const uint32_t lane = threadIdx.x & 31;
-    uint32_t word = sc << (8 * (lane & 3));
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if (in_pad && (lane & 3) == 0)
-        *reinterpret_cast<uint32_t*>(scales + scale_byte_offset(row, kb, nb >> 2)) = word;
+    uint32_t v = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t w = 0;
+        for (int k = 0; k < ONEPASS_THREADS / 32; ++k) w = max(w, red[k]);
+        atomicMax(&ws[WS_AMAX_BITS], w);
+        __threadfence();
+        const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
+        bool ok = true;
+        if (ticket == gridDim.x - 1) {
+            __threadfence();
+            const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
+            atomicExch(&ws[WS_TICKET], 0u);
+            const float amax = __uint_as_float(bits << 16);
+            *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+            __threadfence();
+            atomicAdd(&ws[WS_GENERATION], 1u);
+        } else {
+            const long long t0 = clock64();
+            while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
+                if (clock64() - t0 > timeout) {
+                    ok = false;
+                    if (status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
+                    break;
+                }
+            }
+        }
+        ok_shared = ok;
+    }
+    __syncthreads();
+    if (!ok_shared) return;
+    const float alpha = *reinterpret_cast<volatile float*>(alpha_out);
+
+    // ---- phase 2: quantize, from the end of the tensor backwards (the
+    // lines phase 1 read last are the likeliest to still be in L2); one
+    // thread per four consecutive blocks of a row and step
+    const uint32_t quads = (uint32_t)(K / 64);
+    const int64_t total = prows * quads;                   // padded rows: their scales are zero
+    const int64_t steps = (total + stride - 1) / stride;
+    const int64_t t0 = (int64_t)blockIdx.x * ONEPASS_THREADS + threadIdx.x;
+    for (int64_t s = steps - 1; s >= 0; --s) {
+        const int64_t g = s * stride + t0;
+        if (g >= total) continue;
+        const uint32_t row = (uint32_t)g / quads, q = (uint32_t)g - row * quads;
+        uint4 v[8];
+        load_quad(x, rows, K, row, q, v);
+        quantize_quad(x, rows, K, row, q, alpha, codes, scales, v);
+    }
+}
+
+cudaError_t launch_quantize_onepass(const void* x, int64_t rows, int64_t K, uint32_t* ws_words, float* alpha_out,
+                                    uint8_t* codes, uint8_t* scales, int* status, long long timeout_cycles,
+                                    cudaStream_t stream) {
+    static int blocks_per_sm[64] = {};
+    static int sms[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int d = dev < 64 ? dev : 63;
+    if (!blocks_per_sm[d]) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm[d], k_quantize_onepass,
+                                                                      ONEPASS_THREADS, 0);
+        if (e != cudaSuccess || blocks_per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int64_t prows = padded_rows(rows);
+    const int64_t need = (prows * (K / 64) + ONEPASS_THREADS - 1) / ONEPASS_THREADS;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)sms[d] * blocks_per_sm[d]));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;     // all blocks resident: the grid barrier needs it
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(ONEPASS_THREADS);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_quantize_onepass, reinterpret_cast<const uint4*>(x), rows, prows, K, ws_words,
+                              alpha_out, reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
 }
 
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
-                        int num_sms, cudaStream_t stream) {
+                        int num_sms, cudaStream_t stream, int* clear, int nclear) {
     const int64_t nvec = numel / 8;
     const int ntail = (int)(numel - nvec * 8);
     const uint16_t* tail = reinterpret_cast<const uint16_t*>(x) + nvec * 8;
-    int64_t want = (nvec + AMAX_THREADS * 4 - 1) / (AMAX_THREADS * 4);
+    int64_t want = (nvec + AMAX_THREADS * 8 - 1) / (AMAX_THREADS * 8);
     int blocks = (int)std::min<int64_t>(std::max<int64_t>(want, 1), (int64_t)num_sms * 4);
     k_amax<<<blocks, AMAX_THREADS, 0, stream>>>(reinterpret_cast<const uint4*>(x), nvec, tail, ntail,
-                                               ws_words, alpha_out);
+                                               ws_words, alpha_out, clear, nclear);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
     const int64_t prows = padded_rows(rows);
-    const int64_t threads = prows * (K / 16);
+    const int64_t threads = prows * (K / 64);
     const int64_t blocks = (threads + QUANT_THREADS - 1) / QUANT_THREADS;
     k_quantize<<<(unsigned)blocks, QUANT_THREADS, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), rows, prows, K, alpha, reinterpret_cast<uint2*>(codes), scales);
+        reinterpret_cast<const uint4*>(x), rows, prows, K, alpha, reinterpret_cast<uint4*>(codes), scales);
     return cudaGetLastError();
 }
 

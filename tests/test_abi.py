@@ -52,7 +52,8 @@ def test_sizes(libmq):
     assert mq.mq_nvfp4_scales_bytes(1, 64) == 128 * 4
     assert mq.mq_nvfp4_scales_bytes(130, 320) == 256 * 20
     assert mq.mq_workspace_bytes() == 256
-    assert mq.mq_linear_w4a4_workspace_bytes(128, 1024) == 256 + 65536 + 8192
+    # header | readiness flags (1 row tile x 4 K stages, padded to 256 B) | codes | scales
+    assert mq.mq_linear_w4a4_workspace_bytes(128, 1024) == 256 + 256 + 65536 + 8192
 
 
 def test_host_validation_without_gpu(libmq):

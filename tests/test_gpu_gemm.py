@@ -120,6 +120,34 @@ def test_linear_equals_separate_calls_and_oracle():
     assert rel_frobenius(bf16_bits_to_f64(bits(y)), bf16_bits_to_f64(ref["y_bf16"])) <= TOL
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (130, 300, 320), (257, 513, 1024), (700, 1024, 4096),
+                                   (128, 256, 12288), (2100, 768, 2048)])
+@pytest.mark.parametrize("form", ["auto", "1", "2"])
+def test_linear_paths_agree(M, N, K, form, monkeypatch):
+    """The three ways mq_linear_w4a4 can quantize X -- the one-pass
+    cooperative quantizer (default), the tensor-scale + quantize kernels, and
+    quantizer warps inside the GEMM -- give the same Y bit for bit, and the
+    oracle's within tolerance."""
+    if form != "auto":
+        monkeypatch.setenv("MQ_GEMM_FORM", form)
+    x, w = _random_case(M, N, K, seed=M + 3 * N + K, student_t=(M % 2 == 0))
+    qw = mq.quantize(w.to(dev()))
+    xd = x.to(dev())
+    ws = mq.workspace(mq.mq_linear_w4a4_workspace_bytes(M, K), dev())
+    outs = []
+    for path in ("onepass", "split", "ingemm", "onepass"):
+        monkeypatch.setenv("MQ_LINEAR_PATH", path)
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev())
+        mq.mq_linear_w4a4(xd, qw.codes, qw.scales, qw.alpha, N, y, ws)
+        torch.cuda.synchronize()
+        assert mq.mq_read_status(ws) == mq.MQ_OK
+        outs.append(bits(y))
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+    ref = oracle.linear_w4a4(bits(x), bits(w))
+    assert rel_frobenius(bf16_bits_to_f64(outs[0]), bf16_bits_to_f64(ref["y_bf16"])) <= TOL
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("proj", inputs.QWEN3_8B_PROJECTIONS, ids=lambda p: p.name)
 def test_prefill_projection_8k_sampled_rows(proj):
