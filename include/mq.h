@@ -176,6 +176,22 @@ int mq_linear_w4a4_noalloc(const void *x, int64_t M, int64_t K,
  */
 int mq_read_status(void *ws, void *stream, int32_t *device_status);
 
+/*
+ * Failure-detection test hook; the paper has no counterpart.  Runs the
+ * mq_nvfp4_gemm kernel with the loads of the first pipeline stage withheld
+ * and every bounded wait limited to `timeout_cycles` SM clock cycles
+ * (1e5 .. 4e9), so the pipeline stalls on purpose: each waiting role gives
+ * up, the kernel writes MQ_ERR_TIMEOUT into the workspace status word, lets
+ * its own copies land, frees its tensor memory and returns.  No fault, trap
+ * or hang is involved; the CUDA context stays usable and mq_read_status(ws)
+ * then returns MQ_ERR_TIMEOUT.  Arguments as for mq_nvfp4_gemm; `ws` is
+ * required.  y is left undefined.
+ */
+int mq_debug_gemm_stall(const uint8_t *a_codes, const uint8_t *a_scales, const float *alpha_a,
+                        const uint8_t *b_codes, const uint8_t *b_scales, const float *alpha_b,
+                        int64_t M, int64_t N, int64_t K, void *y, void *ws, size_t ws_bytes,
+                        int64_t timeout_cycles, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

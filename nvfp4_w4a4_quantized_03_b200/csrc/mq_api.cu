@@ -198,6 +198,27 @@ int mq_linear_w4a4(const void* x, int64_t M, int64_t K, const uint8_t* w_codes, 
     return cuda_status(mq::launch_gemm(g, sms, s));
 }
 
+int mq_debug_gemm_stall(const uint8_t* a_codes, const uint8_t* a_scales, const float* alpha_a,
+                        const uint8_t* b_codes, const uint8_t* b_scales, const float* alpha_b, int64_t M, int64_t N,
+                        int64_t K, void* y, void* ws, size_t ws_bytes, int64_t timeout_cycles, void* stream) {
+    if (!ws || ws_bytes < mq::WS_HEADER_BYTES) return MQ_ERR_WORKSPACE;
+    if (!aligned16(ws)) return MQ_ERR_ALIGN;
+    if (timeout_cycles < 100000 || timeout_cycles > DEFAULT_TIMEOUT_CYCLES) return MQ_ERR_INVALID_ARG;
+    if (!a_codes || !a_scales || !alpha_a || !b_codes || !b_scales || !alpha_b || !y) return MQ_ERR_INVALID_ARG;
+    int st = check_rows_k(M, K);
+    if (st != MQ_OK) return st;
+    st = check_rows_k(N, K);
+    if (st != MQ_OK) return st;
+    if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(y))
+        return MQ_ERR_ALIGN;
+    int sms = 0;
+    st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    mq::GemmArgs g{a_codes, a_scales, alpha_a, b_codes, b_scales, alpha_b, y, M, N, K,
+                   static_cast<int*>(ws) + mq::WS_STATUS, (long long)timeout_cycles, 1};
+    return cuda_status(mq::launch_gemm(g, sms, static_cast<cudaStream_t>(stream)));
+}
+
 int mq_read_status(void* ws, void* stream, int32_t* device_status) {
     if (!ws || !device_status) return MQ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -291,13 +291,18 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 }
             }
             if (*abort_flag) {
-                // let the copies this thread issued land before the CTA exits
+                // Let the copies this thread issued land before the CTA
+                // releases its shared memory: a stage's scale copies complete
+                // its sf_full barrier by themselves; its code tiles were
+                // issued right after them and get a short grace period (their
+                // `ready` barrier also needs scale-writer arrivals that an
+                // aborted pipeline no longer makes).
                 for (int i = 0; i < C::STAGES; ++i)
-                    if (pending & (1u << i)) {
+                    if (pending & (1u << i))
                         mbar_wait_bounded(&s->sf_full[i], (pending_phase >> i) & 1, p.timeout, nullptr);
-                        if (rank == 0)
-                            mbar_wait_bounded(&s->ready[i], (pending_phase >> i) & 1, p.timeout, nullptr);
-                    }
+                const long long t0 = clock64();
+                while (clock64() - t0 < 200000) {
+                }
             }
         }
     } else if (warp == 1) {
