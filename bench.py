@@ -257,6 +257,7 @@ def run_ours(args, world, rank, local):
     value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
 
     quant = _quantizer_pass(args, work, device, stream)
+    gemm = _gemm_pass(args, work, device, stream)
     e2e = _e2e(args, work, device, stream)
 
     peaks, peaks_src = _peaks()
@@ -272,10 +273,16 @@ def run_ours(args, world, rank, local):
         "fp4_frac_of_nominal_9pf": value / 9000.0,
         "linear_tflops_by_projection": by_proj,
         "quant_gbs": quant["gbs"],
-        "roofline": {"bound": "tensor", "achieved": lin_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": lin_tflops / fp4_peak, "traffic": None,
-                     "kernel": "mq_linear_w4a4 = k_amax + k_gemm<fused> (k_gemm ~0.9 of its time)",
-                     "peak_source": f"{peaks_src}: 4 x bf16_tflops_sustained"},
+        "gemm_tflops_by_projection": gemm["by_proj"],
+        # the dominant kernel: k_gemm, ~0.8 of each linear's time
+        "roofline": {"bound": "tensor", "achieved": gemm["tflops"], "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm["tflops"] / fp4_peak, "traffic": None,
+                     "kernel": "k_gemm (mq_nvfp4_gemm on the four projections, pre-quantized X)",
+                     "flops_per_launch": "2*8192*N*K", "ms_per_launch": gemm["ms_per_launch"],
+                     "peak_source": f"{peaks_src}: 4 x bf16_tflops_sustained (nominal fp4:bf16 = 4)"},
+        "linear_roofline": {"bound": "tensor", "achieved": lin_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                            "frac": lin_tflops / fp4_peak,
+                            "kernel": "mq_linear_w4a4 = k_quantize_onepass + k_gemm"},
         "quant_roofline": {"bound": "hbm", "achieved": quant["gbs"], "peak": hbm, "unit": "GB/s",
                            "frac": quant["gbs"] / hbm, "traffic": None,
                            "kernel": "k_amax + k_quantize (mq_tensor_scale + mq_nvfp4_quantize)",
@@ -317,6 +324,44 @@ def _quantizer_pass(args, work, device, stream):
     ms = s.elapsed_time(e) / steps
     elems = sum(x.numel() for x, _, _ in bufs)
     return {"gbs": elems * 4.5625 / (ms / 1e3) / 1e9, "ms": ms}
+
+
+def _gemm_pass(args, work, device, stream):
+    """k_gemm alone: mq_nvfp4_gemm of the quantized X against the quantized
+    weight, the launch mq_linear_w4a4 makes after quantizing X.  CUDA events
+    around every launch on the launching stream."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    bufs = []
+    for t in work:
+        qx = mq.quantize(t["x"])
+        bufs.append((t, qx, mq.workspace(mq.mq_workspace_bytes(), device)))
+
+    def run(ev=None):
+        for i, (t, qx, ws) in enumerate(bufs):
+            if ev is not None:
+                ev[i][0].record(stream)
+            mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, t["qw"].codes, t["qw"].scales, t["qw"].alpha,
+                             TOKENS, t["p"].N, t["p"].K, t["y"], ws, stream)
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(3):
+        run()
+    steps = max(5, min(args.steps, 50))
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in bufs] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for k in range(steps):
+        run(evs[k])
+    torch.cuda.synchronize()
+    for _, _, ws in bufs:
+        assert mq.mq_read_status(ws) == mq.MQ_OK
+    by_proj, total_ms = {}, 0.0
+    for i, (t, _, _) in enumerate(bufs):
+        ms_i = sum(ev[i][0].elapsed_time(ev[i][1]) for ev in evs) / steps
+        total_ms += ms_i
+        by_proj[t["p"].name] = 2.0 * TOKENS * t["p"].N * t["p"].K / (ms_i / 1e3) / 1e12
+    return {"tflops": _flops_per_step() / (total_ms / 1e3) / 1e12, "by_proj": by_proj,
+            "ms_per_launch": total_ms / len(bufs)}
 
 
 def _e2e(args, work, device, stream):

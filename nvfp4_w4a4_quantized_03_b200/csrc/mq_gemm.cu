@@ -50,6 +50,7 @@
 
 #include <algorithm>
 #include <cstdlib>
+#include <cstring>
 
 #include "mq_internal.h"
 #include "mq_nvfp4.cuh"
@@ -90,11 +91,16 @@ struct Cfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t SF_COLS_PER_STAGE = 12 * NKB;   // per MMA: A 4 columns, B 8 columns
     static constexpr uint32_t SFB_OFF = 4 * NKB;              // B scales after the A scales of a stage
-    static constexpr int SMEM_STAGES = (SMEM_LIMIT - 1024 - BARRIER_BYTES) / STAGE_BYTES;
+    // Y leaves through shared memory and TMA stores in the pair form: one
+    // 32-row x 64-column bf16 box (4 KB, 128-byte swizzle) per epilogue warp
+    static constexpr bool TMA_STORE = PAIR == 2;
+    static constexpr int EPI_BOX_BYTES = 32 * 64 * 2;
+    static constexpr int EPI_BYTES = TMA_STORE ? EPI_WARPS * EPI_BOX_BYTES : 0;
+    static constexpr int SMEM_STAGES = (SMEM_LIMIT - 1024 - BARRIER_BYTES - EPI_BYTES) / STAGE_BYTES;
     static constexpr int TMEM_STAGES = (TMEM_COLS - SF_COL) / SF_COLS_PER_STAGE;
     static constexpr int STAGES = SMEM_STAGES < TMEM_STAGES ? (SMEM_STAGES < MAX_STAGES ? SMEM_STAGES : MAX_STAGES)
                                                             : (TMEM_STAGES < MAX_STAGES ? TMEM_STAGES : MAX_STAGES);
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + BARRIER_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*align*/ + BARRIER_BYTES;
     static constexpr int TILE_M = BM * PAIR;
     static constexpr uint32_t SWIZZLE = ROW_BYTES == 128 ? 2 : 4;     // descriptor layout: 128B / 64B swizzle
     static constexpr uint32_t SBO = 8 * ROW_BYTES;                    // 8-row swizzle atom
@@ -123,6 +129,9 @@ struct Params {
     int* status;
     long long timeout;
     int fault_skip_first_load;
+    int y_tma;               // Y is written by TMA stores (tmap_y is valid)
+    int pf_dist;             // L2 prefetch distance in stages (0: none)
+    int hints;               // bit 1: evict-first stores of Y
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
     uint8_t* x_codes;        // fused linear: where A's codes are written
     uint8_t* x_scales;       // fused linear: where A's scales are written
@@ -171,7 +180,8 @@ __device__ __forceinline__ void commit_to_all(uint64_t* bar) {
 
 template <int PAIR, int BK, bool QUANT>
 __global__ void __launch_bounds__(THREADS, 1)
-k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, Params p) {
+k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+       const __grid_constant__ CUtensorMap tmap_y, Params p) {
     using C = Cfg<PAIR, BK>;
     constexpr int NKB = C::NKB;
     constexpr int A_BYTES = C::A_BYTES;
@@ -182,7 +192,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
     static_assert(sizeof(Smem) <= BARRIER_BYTES, "barrier area");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Smem* s = reinterpret_cast<Smem*>(base + C::STAGES * C::STAGE_BYTES);
+    uint8_t* epi_stage = base + C::STAGES * C::STAGE_BYTES;          // 1024-byte aligned
+    Smem* s = reinterpret_cast<Smem*>(epi_stage + C::EPI_BYTES);
     auto stage_a = [&](int st) { return base + st * C::STAGE_BYTES; };
     auto stage_b = [&](int st) { return base + st * C::STAGE_BYTES + A_BYTES; };
     auto stage_sfa = [&](int st) { return base + st * C::STAGE_BYTES + A_BYTES + C::B_BYTES; };
@@ -209,6 +220,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
+        if (C::TMA_STORE && p.y_tma) prefetch_tmap(&tmap_y);
     }
     if (warp == 1) {
         if (PAIR == 2) {
@@ -286,6 +298,19 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         else tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
                         pending |= 1u << st;
                         pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
+                    }
+                    if (p.pf_dist > 0) {
+                        // warm L2 with the stage pf_dist ahead (of this tile or a later one)
+                        int kt2 = kt + p.pf_dist, tile2 = tile;
+                        while (kt2 >= p.k_stages) { kt2 -= p.k_stages; tile2 += units; }
+                        if (tile2 < p.tiles) {
+                            int mb2, nb2;
+                            tile_coords(tile2, p, mb2, nb2);
+                            const int arow2 = mb2 * C::TILE_M + (int)rank * BM;
+                            const int brow2 = nb2 * BN + (int)rank * C::B_ROWS;
+                            tma_prefetch_2d(&tmap_b, kt2 * C::ROW_BYTES, brow2);
+                            if (!QUANT) tma_prefetch_2d(&tmap_a, kt2 * C::ROW_BYTES, arow2);
+                        }
                     }
                     if (++st == C::STAGES) { st = 0; phase ^= 1; }
                 }
@@ -470,7 +495,60 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             const int row = mb * C::TILE_M + (int)rank * BM + quad * 32 + lane;
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
             const int colh = nb * BN + half * 128;
-            if (vec_ok && nb * BN + BN <= p.N) {
+            if (C::TMA_STORE && p.y_tma) {
+                // This warp's 32 x 128 block of the accumulator leaves as two
+                // 32 x 64 bf16 boxes through the warp's staging buffer (TMA
+                // stores clip rows >= M and columns >= N).  Columns 0-63 are
+                // staged while draining; TMEM is handed back once all 128
+                // columns are in registers or shared memory.
+                uint8_t* box = epi_stage + (warp - FIRST_EPI_WARP) * C::EPI_BOX_BYTES;
+                const uint32_t box_row = smem_u32(box) + lane * 128;
+                const int row0 = mb * C::TILE_M + (int)rank * BM + quad * 32;
+                // 16-byte chunk j of a 128-byte box row sits at chunk j ^ (row % 8)
+                auto stage_chunk = [&](int j, const uint32_t* v) {
+                    st_shared_v4(box_row + ((j ^ (lane & 7)) << 4), v[0], v[1], v[2], v[3]);
+                };
+                auto issue = [&](int h) {
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0 && row0 < p.M && colh + h * 64 < p.N) {
+                        tma_store_2d(&tmap_y, box, colh + h * 64, row0);
+                        bulk_commit_group();
+                    }
+                };
+                if (lane == 0) bulk_wait_group_read0();         // the previous tile's box has been read
+                __syncwarp();
+                uint32_t hi[2][16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        pk[j] = cvt_bf16x2(__fmul_rn(__uint_as_float(r[2 * j + 1]), ab),
+                                           __fmul_rn(__uint_as_float(r[2 * j]), ab));
+                    if (c < 2) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) stage_chunk(c * 4 + q, pk + 4 * q);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) hi[c - 2][j] = pk[j];
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
+                issue(0);
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) stage_chunk(c * 4 + q, hi[c] + 4 * q);
+                issue(1);
+            } else if (!C::TMA_STORE && vec_ok && nb * BN + BN <= p.N) {
                 // Whole tile inside Y: drain this warp's 32 x 128 block of the
                 // accumulator (scaled and rounded to bf16 on the way), hand TMEM
                 // back so the next tile's MMAs overlap the stores, then store.
@@ -490,12 +568,25 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
                 if (row < p.M) {
                     uint4* d4 = reinterpret_cast<uint4*>(p.y + (int64_t)row * p.N + colh);
+                    if (p.hints & 2) {
+                        // Y is not read again here: let it leave L2 before A and B
+                        const uint64_t pol = policy_evict_first();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                        for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            d4[c * 4 + j] = make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
-                                                       packed[c][4 * j + 2], packed[c][4 * j + 3]);
+                            for (int j = 0; j < 4; ++j)
+                                st_global_hint(d4 + c * 4 + j,
+                                               make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
+                                                          packed[c][4 * j + 2], packed[c][4 * j + 3]),
+                                               pol);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                d4[c * 4 + j] = make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
+                                                           packed[c][4 * j + 2], packed[c][4 * j + 3]);
+                    }
                 }
             } else {
                 // Ragged right edge (or N not a multiple of 8): one 32-column
@@ -525,6 +616,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         }
     }
 
+    if (C::TMA_STORE && warp >= FIRST_EPI_WARP && lane == 0) bulk_wait_group0();
     __syncwarp();   // reconverge the single-lane roles before the block barrier
     tc_fence_before();
     __syncthreads();
@@ -539,6 +631,13 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
 }  // namespace gemm
 
 // ---------------------------------------------------------------- host side
+static int env_int(const char* name, int lo, int hi, int dflt) {
+    const char* v = getenv(name);
+    if (!v) return dflt;
+    const int x = atoi(v);
+    return (x >= lo && x <= hi) ? x : dflt;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -569,6 +668,20 @@ static bool make_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, 
                CU_TENSOR_MAP_INTERLEAVE_NONE,
                box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor [M, N] for the epilogue's TMA stores: 32-row x 64-column
+// boxes in the 128-byte swizzle.  Needs N % 8 == 0 (16-byte row pitch).
+static bool make_y_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || N % 8 != 0 || (reinterpret_cast<uintptr_t>(y) & 15u)) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(N * 2)};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 namespace {
@@ -610,10 +723,12 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
         }
         fs.attr_set = true;
     }
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, my;
     if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM, C::ROW_BYTES) ||
         !make_code_map(&mb, a.b_codes, a.N, a.K, C::B_ROWS, C::ROW_BYTES))
         return cudaErrorInvalidValue;
+    memset(&my, 0, sizeof(my));
+    const bool y_tma = C::TMA_STORE && env_int("MQ_GEMM_YTMA", 0, 1, 1) && make_y_map(&my, a.y, a.M, a.N);
     Params p{};
     p.a_scales = a.a_scales;
     p.b_scales = a.b_scales;
@@ -634,6 +749,9 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.status = a.status;
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
+    p.y_tma = y_tma ? 1 : 0;
+    p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
+    p.hints = env_int("MQ_GEMM_HINTS", 0, 3, 0);
     p.x = static_cast<const uint16_t*>(a.x);
     p.x_codes = const_cast<uint8_t*>(a.a_codes);
     p.x_scales = const_cast<uint8_t*>(a.a_scales);
@@ -662,7 +780,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = nattr;
-    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, p);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, my, p);
 }
 
 int env_choice(const char* name, int a, int b, int dflt) {
