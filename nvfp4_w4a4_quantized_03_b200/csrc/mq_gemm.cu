@@ -72,7 +72,7 @@ constexpr int THREADS = (FIRST_EPI_WARP + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = BN;                     // stage st: SF_COL + st * SF_COLS_PER_STAGE
-constexpr int GROUP_M = 8;                          // tile raster: M-blocks per group
+constexpr int GROUP_M = 32;                         // tile raster: default M-blocks per group
 constexpr int MAX_STAGES = 10;
 constexpr int BARRIER_BYTES = 512;
 constexpr int SMEM_LIMIT = 232448;                  // dynamic shared memory per block on sm_100
@@ -132,6 +132,8 @@ struct Params {
     int y_tma;               // Y is written by TMA stores (tmap_y is valid)
     int pf_dist;             // L2 prefetch distance in stages (0: none)
     int hints;               // bit 1: evict-first stores of Y
+    int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
+    int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
     uint8_t* x_codes;        // fused linear: where A's codes are written
     uint8_t* x_scales;       // fused linear: where A's scales are written
@@ -152,9 +154,9 @@ struct Smem {
 };
 
 __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
-    const int group = GROUP_M * p.n_blocks;
-    const int first_m = (tile / group) * GROUP_M;
-    const int gm = min(GROUP_M, p.m_blocks - first_m);
+    const int group = p.group_m * p.n_blocks;
+    const int first_m = (tile / group) * p.group_m;
+    const int gm = min(p.group_m, p.m_blocks - first_m);
     const int in = tile % group;
     mb = first_m + in % gm;
     nb = in / gm;
@@ -312,7 +314,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             if (!QUANT) tma_prefetch_2d(&tmap_a, kt2 * C::ROW_BYTES, arow2);
                         }
                     }
-                    if (++st == C::STAGES) { st = 0; phase ^= 1; }
+                    if (++st == p.stages) { st = 0; phase ^= 1; }
                 }
             }
             if (*abort_flag) {
@@ -341,32 +343,54 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     break;
                 }
                 tc_fence_after();
-                bool ok = true;
-                for (int kt = 0; kt < p.k_stages; ++kt) {
+                // The tensor pipe queues about one MMA behind the running one,
+                // so the gap between the last MMA of a stage and the first of
+                // the next must stay short: the wait for the next stage's
+                // barrier is taken while the stage's last MMAs are still queued.
+                bool ok = mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag);
+                tc_fence_after();
+                for (int kt = 0; ok && kt < p.k_stages; ++kt) {
                     // the stage's codes are in shared memory and its scales in TMEM
-                    if (!mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag)) {
-                        raise_abort(s, p);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
                     const int nkb = min(NKB, p.kblocks - kt * NKB);
-                    const uint32_t a0 = smem_u32(stage_a(st)), b0 = smem_u32(stage_b(st));
+                    const int nst = st + 1 == p.stages ? 0 : st + 1;
+                    const uint32_t nphase = st + 1 == p.stages ? phase ^ 1 : phase;
+                    const bool more = kt + 1 < p.k_stages;
+                    // descriptors of the stage's first K step; the next steps
+                    // start MMA_K / 2 bytes further (address field in 16-byte units)
+                    const uint64_t ad0 = smem_desc(smem_u32(stage_a(st)), 16, C::SBO, C::SWIZZLE);
+                    const uint64_t bd0 = smem_desc(smem_u32(stage_b(st)), 16, C::SBO, C::SWIZZLE);
                     const uint32_t sf = tmem + SF_COL + st * SF_COLS_PER_STAGE;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        const uint64_t ad = smem_desc(a0 + kb * (MMA_K / 2), 16, C::SBO, C::SWIZZLE);
-                        const uint64_t bd = smem_desc(b0 + kb * (MMA_K / 2), 16, C::SBO, C::SWIZZLE);
+                    auto mma = [&](int kb) {
+                        const uint64_t step = (uint64_t)(kb * (MMA_K / 2) >> 4);
                         if (PAIR == 2)
-                            mma_mxf4nvf4_pair(tmem + ACC_COL, ad, bd, C::IDESC, sf + kb * 4, sf + SFB_OFF + kb * 8,
-                                              (kt | kb) != 0);
+                            mma_mxf4nvf4_pair(tmem + ACC_COL, ad0 + step, bd0 + step, C::IDESC, sf + kb * 4,
+                                              sf + SFB_OFF + kb * 8, (kt | kb) != 0);
                         else
-                            mma_mxf4nvf4(tmem + ACC_COL, ad, bd, C::IDESC, sf + kb * 4, sf + SFB_OFF + kb * 8,
-                                         (kt | kb) != 0);
+                            mma_mxf4nvf4(tmem + ACC_COL, ad0 + step, bd0 + step, C::IDESC, sf + kb * 4,
+                                         sf + SFB_OFF + kb * 8, (kt | kb) != 0);
+                    };
+                    bool next_ok = true;
+                    if (nkb == NKB) {
+                        // a full stage: no branch between two MMAs (one measured
+                        // ~30% lower tensor-pipe throughput)
+#pragma unroll
+                        for (int kb = 0; kb < NKB - 1; ++kb) mma(kb);
+                        if (more) next_ok = mbar_wait_bounded(&s->ready[nst], nphase, p.timeout, abort_flag);
+                        mma(NKB - 1);
+                    } else {
+                        for (int kb = 0; kb < nkb; ++kb) mma(kb);
+                        if (more) next_ok = mbar_wait_bounded(&s->ready[nst], nphase, p.timeout, abort_flag);
                     }
                     commit_to_all<PAIR>(&s->empty[st]);
-                    if (++st == C::STAGES) { st = 0; phase ^= 1; }
+                    st = nst;
+                    phase = nphase;
+                    if (!next_ok) ok = false;
+                    tc_fence_after();
                 }
-                if (!ok) break;
+                if (!ok) {
+                    raise_abort(s, p);
+                    break;
+                }
                 commit_to_all<PAIR>(&s->acc_full);
                 acc_phase ^= 1;
             }
@@ -380,13 +404,13 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         if constexpr (QUANT) {
             // A unit is 32 rows x one K stage (BK elements, BK / 16 blocks per
             // row).  Units are numbered in the order the tile raster consumes
-            // them: raster group of GROUP_M tile rows, then K stage, then
+            // them: raster group of group_m tile rows, then K stage, then
             // 32-row slab; unit u goes to quantizer warp u mod (all warps).
             static_assert(BK == 256, "the fused quantizer maps one lane to each of a row's 16 blocks");
             const int qw = blockIdx.x * QUANT_WARPS + (warp - FIRST_Q_WARP);
             const int nqw = gridDim.x * QUANT_WARPS;
             const int slabs = p.a_row_tiles * 4;
-            const int slabs_per_group = GROUP_M * C::TILE_M / 32;
+            const int slabs_per_group = p.group_m * C::TILE_M / 32;
             const int64_t per_group = (int64_t)slabs_per_group * p.k_stages;
             const int64_t units = (int64_t)slabs * p.k_stages;
             const float alpha = *p.alpha_a;
@@ -453,21 +477,35 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             for (int kt = 0; kt < p.k_stages; ++kt) {
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s->sf_full[st], phase, p.timeout, abort_flag));
                 if (!ok) break;
-                const int nkb = min(NKB, p.kblocks - kt * NKB);
                 const uint8_t* sfa = stage_sfa(st) + lane * 16;
                 const uint8_t* sfb = stage_sfb(st) + lane * 16;
                 const uint32_t t = tmem + ((uint32_t)(quad * 32) << 16) + SF_COL + st * SF_COLS_PER_STAGE;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    tmem_st_32x32b_x4(t + kb * 4, *reinterpret_cast<const uint4*>(sfa + kb * 512));
-                    tmem_st_32x32b_x4(t + SFB_OFF + kb * 8, *reinterpret_cast<const uint4*>(sfb + kb * 512));
-                    tmem_st_32x32b_x4(t + SFB_OFF + kb * 8 + 4,
-                                      *reinterpret_cast<const uint4*>(sfb + SFB_BYTES / 2 + kb * 512));
+                // The stage's 12 NKB scale columns are contiguous in TMEM: A's
+                // (4 per MMA), then B's (8 per MMA).  All shared-memory reads
+                // first, then one store per operand.  In a K-tail stage the
+                // columns past the last MMA get stale bytes that nothing reads.
+                uint32_t va[4 * NKB], vb[8 * NKB];
+#pragma unroll
+                for (int kb = 0; kb < NKB; ++kb) {
+                    const uint4 a4 = *reinterpret_cast<const uint4*>(sfa + kb * 512);
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + kb * 512);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + SFB_BYTES / 2 + kb * 512);
+                    va[4 * kb] = a4.x; va[4 * kb + 1] = a4.y; va[4 * kb + 2] = a4.z; va[4 * kb + 3] = a4.w;
+                    vb[8 * kb] = b0.x; vb[8 * kb + 1] = b0.y; vb[8 * kb + 2] = b0.z; vb[8 * kb + 3] = b0.w;
+                    vb[8 * kb + 4] = b1.x; vb[8 * kb + 5] = b1.y; vb[8 * kb + 6] = b1.z; vb[8 * kb + 7] = b1.w;
+                }
+                if constexpr (NKB == 4) {
+                    tmem_st_32x32b_x16(t, va);
+                    tmem_st_32x32b_x32(t + SFB_OFF, vb);
+                } else {
+                    tmem_st_32x32b_x8(t, va);
+                    tmem_st_32x32b_x16(t + SFB_OFF, vb);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_leader<PAIR>(&s->ready[st]);
-                if (++st == C::STAGES) { st = 0; phase ^= 1; }
+                if (++st == p.stages) { st = 0; phase ^= 1; }
             }
             if (!ok) {
                 if (lane == 0) raise_abort(s, p);
@@ -752,6 +790,8 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.y_tma = y_tma ? 1 : 0;
     p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
     p.hints = env_int("MQ_GEMM_HINTS", 0, 3, 0);
+    p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
+    p.stages = env_int("MQ_GEMM_STAGES", 2, C::STAGES, C::STAGES);
     p.x = static_cast<const uint16_t*>(a.x);
     p.x_codes = const_cast<uint8_t*>(a.a_codes);
     p.x_scales = const_cast<uint8_t*>(a.a_scales);
