@@ -34,6 +34,25 @@ METRIC = "W4A4 NVFP4 linear TFLOPS (quant+GEMM) & % of B200 FP4 peak; quant GB/s
 WORKLOAD = "qwen3-8b prefill projections (qkv, o, gate_up, down) at 8192 tokens, NVFP4 W4A4"
 
 
+def _gemm_traffic():
+    """DRAM bytes per k_gemm launch (mean over the four projections) from the
+    committed ncu capture, or None once the kernel's sources have changed
+    since the capture (the counters would describe another kernel)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "k_gemm_dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != rec["sources_sha256_16"]:
+        return None
+    return rec["mean_per_launch_bytes"]
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -276,7 +295,8 @@ def run_ours(args, world, rank, local):
         "gemm_tflops_by_projection": gemm["by_proj"],
         # the dominant kernel: k_gemm, ~0.8 of each linear's time
         "roofline": {"bound": "tensor", "achieved": gemm["tflops"], "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm["tflops"] / fp4_peak, "traffic": None,
+                     "frac": gemm["tflops"] / fp4_peak, "traffic": _gemm_traffic(),
+                     "traffic_unit": "bytes per launch (mean of the four projections; ncu dram read+write)",
                      "kernel": "k_gemm (mq_nvfp4_gemm on the four projections, pre-quantized X)",
                      "flops_per_launch": "2*8192*N*K", "ms_per_launch": gemm["ms_per_launch"],
                      "peak_source": f"{peaks_src}: 4 x bf16_tflops_sustained (nominal fp4:bf16 = 4)"},
