@@ -131,7 +131,7 @@ struct Params {
     int fault_skip_first_load;
     int y_tma;               // Y is written by TMA stores (tmap_y is valid)
     int pf_dist;             // L2 prefetch distance in stages (0: none)
-    int hints;               // bit 1: evict-first stores of Y
+    int hints;               // bit 1: evict-first stores of Y (register path); bit 2: same for the TMA stores
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
     int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
@@ -267,22 +267,26 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         skip = false;
                     } else {
                         const int64_t ka = (int64_t)kt * NKB;              // first k-atom of the stage
-                        // B's block scales and codes first: they never wait
-                        mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
-                        for (int rt = 0; rt < 2; ++rt) {
-                            const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
-                            bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
-                                      p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
-                        }
+                        // The code tiles first: they take longest to land (the
+                        // scales need less than half as long, copy and TMEM
+                        // store included).
                         uint32_t bar0 = 0;
                         if (PAIR == 2) {
                             // both CTAs' code tiles complete on CTA 0's barrier
                             if (rank == 0) mbar_arrive_expect_tx(&s->ready[st], 2 * (A_BYTES + C::B_BYTES));
                             bar0 = mapa_shared(smem_u32(&s->ready[st]), 0);
                             tma_load_2d_pair(stage_b(st), &tmap_b, bar0, kt * C::ROW_BYTES, brow);
+                            if (!QUANT) tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
                         } else {
                             mbar_arrive_expect_tx(&s->ready[st], A_BYTES + C::B_BYTES);
                             tma_load_2d(stage_b(st), &tmap_b, &s->ready[st], kt * C::ROW_BYTES, brow);
+                            if (!QUANT) tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
+                        }
+                        mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
+                        for (int rt = 0; rt < 2; ++rt) {
+                            const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
+                            bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
+                                      p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
                         }
                         if (QUANT && arow / 128 < p.a_row_tiles) {
                             // A's block (arow, kt) is written by quantizer warps (of any CTA)
@@ -296,8 +300,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             fence_proxy_async_global();
                         }
                         bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
-                        if (PAIR == 2) tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
-                        else tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
+                        if (QUANT) {
+                            if (PAIR == 2) tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
+                            else tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
+                        }
                         pending |= 1u << st;
                         pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
                     }
@@ -536,9 +542,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             if (C::TMA_STORE && p.y_tma) {
                 // This warp's 32 x 128 block of the accumulator leaves as two
                 // 32 x 64 bf16 boxes through the warp's staging buffer (TMA
-                // stores clip rows >= M and columns >= N).  Columns 0-63 are
-                // staged while draining; TMEM is handed back once all 128
-                // columns are in registers or shared memory.
+                // stores clip rows >= M and columns >= N).  The four 32-column
+                // TMEM loads are double-buffered (chunk c + 1 loads while chunk
+                // c is scaled, rounded and staged); TMEM goes back to the MMA
+                // thread as soon as the last load has landed.
                 uint8_t* box = epi_stage + (warp - FIRST_EPI_WARP) * C::EPI_BOX_BYTES;
                 const uint32_t box_row = smem_u32(box) + lane * 128;
                 const int row0 = mb * C::TILE_M + (int)rank * BM + quad * 32;
@@ -550,34 +557,39 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0 && row0 < p.M && colh + h * 64 < p.N) {
-                        tma_store_2d(&tmap_y, box, colh + h * 64, row0);
+                        if (p.hints & 4) tma_store_2d_hint(&tmap_y, box, colh + h * 64, row0, policy_evict_first());
+                        else tma_store_2d(&tmap_y, box, colh + h * 64, row0);
                         bulk_commit_group();
                     }
                 };
-                if (lane == 0) bulk_wait_group_read0();         // the previous tile's box has been read
-                __syncwarp();
-                uint32_t hi[2][16];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(taddr + c * 32, r);
-                    tmem_ld_wait();
-                    uint32_t pk[16];
+                auto convert = [&](const uint32_t (&r)[32], uint32_t (&pk)[16]) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         pk[j] = cvt_bf16x2(__fmul_rn(__uint_as_float(r[2 * j + 1]), ab),
                                            __fmul_rn(__uint_as_float(r[2 * j]), ab));
-                    if (c < 2) {
+                };
+                if (lane == 0) bulk_wait_group_read0();         // the previous tile's box has been read
+                __syncwarp();
+                uint32_t ra[32], rb[32], pk[16], hi[2][16];
+                tmem_ld_32x32b_x32(taddr, ra);
+                tmem_ld_wait_regs(ra);
+                tmem_ld_32x32b_x32(taddr + 32, rb);
+                convert(ra, pk);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) stage_chunk(c * 4 + q, pk + 4 * q);
-                    } else {
+                for (int q = 0; q < 4; ++q) stage_chunk(q, pk + 4 * q);
+                tmem_ld_wait_regs(rb);
+                tmem_ld_32x32b_x32(taddr + 64, ra);
+                convert(rb, pk);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) hi[c - 2][j] = pk[j];
-                    }
-                }
+                for (int q = 0; q < 4; ++q) stage_chunk(4 + q, pk + 4 * q);
+                tmem_ld_wait_regs(ra);
+                tmem_ld_32x32b_x32(taddr + 96, rb);
+                convert(ra, hi[0]);
+                tmem_ld_wait_regs(rb);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
+                convert(rb, hi[1]);
                 issue(0);
                 if (lane == 0) bulk_wait_group_read0();
                 __syncwarp();
@@ -789,7 +801,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.fault_skip_first_load = a.fault_skip_first_load;
     p.y_tma = y_tma ? 1 : 0;
     p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
-    p.hints = env_int("MQ_GEMM_HINTS", 0, 3, 0);
+    p.hints = env_int("MQ_GEMM_HINTS", 0, 7, 0);
     p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
     p.stages = env_int("MQ_GEMM_STAGES", 2, C::STAGES, C::STAGES);
     p.x = static_cast<const uint16_t*>(a.x);
