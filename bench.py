@@ -278,6 +278,9 @@ def run_ours(args, world, rank, local):
     quant = _quantizer_pass(args, work, device, stream)
     gemm = _gemm_pass(args, work, device, stream)
     e2e = _e2e(args, work, device, stream)
+    del work
+    torch.cuda.empty_cache()
+    sequence = None if args.no_sequence else _prefill_sequence(args, device)
 
     peaks, peaks_src = _peaks()
     fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]        # nominal fp4 : bf16 = 9 : 2.25
@@ -310,6 +313,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 8 * args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "prefill_sequence": sequence,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
@@ -384,6 +388,37 @@ def _gemm_pass(args, work, device, stream):
             "ms_per_launch": total_ms / len(bufs)}
 
 
+def _prefill_sequence(args, device):
+    """The 36-layer decoder stack's prefill linears at 131072 tokens (four
+    Qwen3-8B-shaped projections per layer, fixed activations, weights
+    N(0, 0.02) quantized offline), recorded once as a CUDA graph and replayed;
+    CUDA events around each replay."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    from nvfp4_w4a4_quantized_03_b200.sequence import PrefillSequence
+    layers, tokens = 36, 131072
+    seq = PrefillSequence(layers, tokens, device)
+    seq.capture()
+    seq.replay()                      # warm-up
+    torch.cuda.synchronize()
+    reps = 3
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    stream = torch.cuda.current_stream()
+    for e0, e1 in evs:
+        e0.record(stream)
+        seq.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    assert seq.status() == mq.MQ_OK
+    ms = min(e0.elapsed_time(e1) for e0, e1 in evs)
+    out = {"workload": f"{layers} layers x (qkv, o, gate_up, down) at {tokens} tokens, one CUDA graph",
+           "tflops": seq.flops() / (ms / 1e3) / 1e12, "ms": ms, "ms_per_layer": ms / layers,
+           "tflop_per_layer": seq.flops() / layers / 1e12, "graph_kernel_launches": 2 * 4 * layers,
+           "replays_timed": reps, "timing": "best of the timed replays"}
+    del seq
+    torch.cuda.empty_cache()
+    return out
+
+
 def _e2e(args, work, device, stream):
     """Pinned host X -> device, mq_linear_w4a4, device -> pinned host Y, per step."""
     from nvfp4_w4a4_quantized_03_b200 import mq
@@ -422,6 +457,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sequence", action="store_true",
+                    help="skip the 36-layer x 131072-token prefill-sequence figure")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world, rank, local = _dist()
