@@ -23,6 +23,10 @@ constexpr size_t WS_HEADER_BYTES = 256;
 __host__ __device__ inline int64_t scale_atom_cols(int64_t K) { return (K / 16 + 3) / 4; }
 __host__ __device__ inline int64_t padded_rows(int64_t rows) { return (rows + 127) / 128 * 128; }
 
+// Tensor map of a bf16 [rows, K] tensor for TMA loads of box_rows x 64-element
+// boxes in the 128-byte swizzle (rows past the end read as zero).
+bool make_bf16_tile_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K, int box_rows);
+
 // Launchers (enqueue on `stream`, no synchronisation).
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
                         int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0);

@@ -18,6 +18,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "mq_internal.h"
 #include "mq_nvfp4.cuh"
@@ -120,6 +121,183 @@ k_quantize(const uint4* __restrict__ x, int64_t rows, int64_t prows, int64_t K,
     quantize_quad(x, rows, K, row, q, __ldg(alpha_p), codes, scales, v);
 }
 
+// ---------------------------------------------------------------------------
+// k_quantize_tiles: the same quantization with X brought into shared memory
+// by TMA, 256 rows x 64 elements (32 KB) per box in the 128-byte swizzle.
+// Thread t quantizes row t of a box (four blocks, one scale word) from its
+// 128-byte row of the box; the swizzle puts the 16-byte chunk j of row t at
+// chunk j ^ (t % 8), so the eight 16-byte shared-memory reads of a warp are
+// conflict-free.  A ring of QT_STAGES boxes per CTA keeps the loads in
+// flight while the previous box is quantized.  (Loading the same data with
+// eight 16-byte global loads per thread measured the L1 at 90% of its
+// throughput: every warp-wide load touched 32 cache lines.)
+constexpr int QT_THREADS = 256;
+constexpr int QT_ROWS = 256;
+constexpr int QT_STAGES = 3;
+constexpr int QT_BOX_BYTES = QT_ROWS * 128;
+constexpr int QT_SMEM = QT_STAGES * QT_BOX_BYTES + 1024;
+
+__global__ void __launch_bounds__(QT_THREADS, 2)
+k_quantize_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
+                 const float* __restrict__ alpha_p, uint4* __restrict__ codes, uint8_t* __restrict__ scales) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[QT_STAGES];
+    const int64_t kgroups = K / 64;
+    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < QT_STAGES; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
+        prefetch_tmap(&xmap);
+    }
+    __syncthreads();
+    auto issue = [&](int64_t t, int st) {
+        mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
+        tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
+                    (int32_t)(t / kgroups) * QT_ROWS);
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < QT_STAGES; ++i)
+            if (blockIdx.x + (int64_t)i * gridDim.x < ntiles) issue(blockIdx.x + (int64_t)i * gridDim.x, i);
+    const float alpha = __ldg(alpha_p);
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+        const int st = it % QT_STAGES;
+        // the box's bytes landed (bounded: a copy that never lands ends the
+        // block rather than hanging it)
+        if (!mbar_wait_bounded(&full[st], (uint32_t)(it / QT_STAGES) & 1, 4000000000LL, nullptr)) break;
+        const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
+        const uint32_t kg = (uint32_t)(t % kgroups);
+        if (row < prows) {
+            const uint8_t* src = base + st * QT_BOX_BYTES + threadIdx.x * 128;
+            uint4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
+            quantize_quad(nullptr, rows, K, (uint32_t)row, kg, alpha, codes, scales, v);
+        }
+        __syncthreads();     // every thread is done with this box
+        if (threadIdx.x == 0 && t + (int64_t)QT_STAGES * gridDim.x < ntiles) issue(t + (int64_t)QT_STAGES * gridDim.x, st);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// k_quantize_onepass_tiles: alpha_x and the codes/scales of X in one
+// cooperative launch, X streamed through the same TMA ring of 256 x 64
+// boxes as k_quantize_tiles.  Each block takes the boxes t = block, block +
+// grid, ... ; "items" 0..n-1 are those boxes in order (phase 1: max |x|),
+// items n..2n-1 the same boxes in reverse order (phase 2: quantize), so the
+// boxes read last in phase 1 (the likeliest to be in L2) are read first in
+// phase 2, and the first boxes of phase 2 are already in flight while the
+// grid barrier between the phases completes.  Rows past the end arrive as
+// zeros, which leave the max unchanged.
+__global__ void __launch_bounds__(QT_THREADS, 2)
+k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
+                         uint32_t* __restrict__ ws, float* __restrict__ alpha_out, uint4* __restrict__ codes,
+                         uint8_t* __restrict__ scales, int* __restrict__ status, long long timeout) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[QT_STAGES];
+    __shared__ uint32_t red[QT_THREADS / 32];
+    __shared__ int ok_shared;
+    __shared__ float alpha_shared;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(&ws[WS_GENERATION]);
+    const int64_t kgroups = K / 64;
+    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
+    const int64_t n = ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;   // boxes of this block
+    auto box_of = [&](int64_t item) -> int64_t {   // item -> box index
+        const int64_t i = item < n ? item : 2 * n - 1 - item;
+        return blockIdx.x + i * gridDim.x;
+    };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < QT_STAGES; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
+        prefetch_tmap(&xmap);
+        ok_shared = 1;
+    }
+    __syncthreads();
+    auto issue = [&](int64_t item) {
+        const int64_t t = box_of(item);
+        const int st = (int)(item % QT_STAGES);
+        mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
+        tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
+                    (int32_t)(t / kgroups) * QT_ROWS);
+    };
+    if (threadIdx.x == 0)
+        for (int64_t i = 0; i < QT_STAGES && i < 2 * n; ++i) issue(i);
+    uint32_t m = 0;
+    float alpha = 0.0f;
+    // end of phase 1: fold this block's max, then the grid barrier (every
+    // block takes part, also one without boxes)
+    auto finish_phase1 = [&]() {
+        uint32_t v = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
+        if (lane == 0) red[warp] = v;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t w = 0;
+            for (int k = 0; k < QT_THREADS / 32; ++k) w = max(w, red[k]);
+            atomicMax(&ws[WS_AMAX_BITS], w);
+            __threadfence();
+            const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
+            if (ticket == gridDim.x - 1) {
+                __threadfence();
+                const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
+                atomicExch(&ws[WS_TICKET], 0u);
+                const float amax = __uint_as_float(bits << 16);
+                *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                __threadfence();
+                atomicAdd(&ws[WS_GENERATION], 1u);
+            } else {
+                const long long t0 = clock64();
+                while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
+                    if (clock64() - t0 > timeout) {
+                        ok_shared = 0;
+                        if (status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
+                        break;
+                    }
+                }
+            }
+            alpha_shared = *reinterpret_cast<volatile float*>(alpha_out);
+        }
+        __syncthreads();
+        alpha = alpha_shared;
+    };
+    if (n == 0) finish_phase1();
+    for (int64_t item = 0; item < 2 * n; ++item) {
+        if (item == n) finish_phase1();
+        const int st = (int)(item % QT_STAGES);
+        // a box that never lands, or a timed-out barrier, ends the block once
+        // its copies in flight have landed (they are waited for below)
+        const bool landed = mbar_wait_bounded(&full[st], (uint32_t)(item / QT_STAGES) & 1, timeout, nullptr);
+        if (!__syncthreads_and(landed && ok_shared)) {     // the same decision in every thread
+            if (threadIdx.x == 0 && status) atomicExch(status, -7);
+            ok_shared = 0;
+            break;
+        }
+        const uint8_t* src = base + st * QT_BOX_BYTES + threadIdx.x * 128;
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
+        if (item < n) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m = absmax_vec(m, v[j]);
+        } else {
+            const int64_t t = box_of(item);
+            const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
+            if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
+        }
+        __syncthreads();     // every thread is done with this box
+        if (threadIdx.x == 0 && item + QT_STAGES < 2 * n) issue(item + QT_STAGES);
+    }
+    // copies still in flight after an early exit land before the block ends
+    if (threadIdx.x == 0 && !ok_shared) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < 200000) {
+        }
+    }
+}
+
 constexpr int ONEPASS_THREADS = 256;
 
 // alpha_x and the codes/scales of a [rows, K] tensor in one launch.  Every
@@ -218,6 +396,35 @@ cudaError_t launch_quantize_onepass(const void* x, int64_t rows, int64_t K, uint
         cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
     }
     const int64_t prows = padded_rows(rows);
+    // the TMA-streamed form (MQ_ONEPASS_TILES=0 selects the per-thread-load form)
+    const char* tv = getenv("MQ_ONEPASS_TILES");
+    CUtensorMap xmap;
+    if (!(tv && tv[0] == '0') && make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) {
+        static int tiles_per_sm[64] = {};
+        if (!tiles_per_sm[d]) {
+            cudaError_t e = cudaFuncSetAttribute(k_quantize_onepass_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 QT_SMEM);
+            if (e != cudaSuccess) return e;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&tiles_per_sm[d], k_quantize_onepass_tiles, QT_THREADS,
+                                                              QT_SMEM);
+            if (e != cudaSuccess || tiles_per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        }
+        // every block resident (grid barrier) and every block owning at least one box
+        const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * tiles_per_sm[d]));
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(QT_THREADS);
+        cfg.dynamicSmemBytes = QT_SMEM;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k_quantize_onepass_tiles, xmap, rows, prows, K, ws_words, alpha_out,
+                                  reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
+    }
     const int64_t need = (prows * (K / 64) + ONEPASS_THREADS - 1) / ONEPASS_THREADS;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)sms[d] * blocks_per_sm[d]));
     cudaLaunchConfig_t cfg = {};
@@ -248,6 +455,26 @@ cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float*
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
     const int64_t prows = padded_rows(rows);
+    const char* tv = getenv("MQ_QUANT_TILES");
+    CUtensorMap xmap;
+    if (!(tv && tv[0] == '0') && make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) {
+        static int sms[64] = {};
+        static bool attr[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const int d = dev < 64 ? dev : 63;
+        if (!attr[d]) {
+            cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
+            cudaError_t e = cudaFuncSetAttribute(k_quantize_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
+            if (e != cudaSuccess) return e;
+            attr[d] = true;
+        }
+        const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, 2 * (int64_t)sms[d]));
+        k_quantize_tiles<<<grid, QT_THREADS, QT_SMEM, stream>>>(xmap, rows, prows, K, alpha,
+                                                                reinterpret_cast<uint4*>(codes), scales);
+        return cudaGetLastError();
+    }
     const int64_t threads = prows * (K / 64);
     const int64_t blocks = (threads + QUANT_THREADS - 1) / QUANT_THREADS;
     k_quantize<<<(unsigned)blocks, QUANT_THREADS, 0, stream>>>(
