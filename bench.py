@@ -281,6 +281,7 @@ def run_ours(args, world, rank, local):
     del work
     torch.cuda.empty_cache()
     sequence = None if args.no_sequence else _prefill_sequence(args, device)
+    decode = None if args.no_sequence else _decode_figure(device)
 
     peaks, peaks_src = _peaks()
     fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]        # nominal fp4 : bf16 = 9 : 2.25
@@ -305,15 +306,16 @@ def run_ours(args, world, rank, local):
                      "peak_source": f"{peaks_src}: 4 x bf16_tflops_sustained (nominal fp4:bf16 = 4)"},
         "linear_roofline": {"bound": "tensor", "achieved": lin_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                             "frac": lin_tflops / fp4_peak,
-                            "kernel": "mq_linear_w4a4 = k_quantize_onepass + k_gemm"},
+                            "kernel": "mq_linear_w4a4 = k_quantize_onepass_tiles + k_gemm"},
         "quant_roofline": {"bound": "hbm", "achieved": quant["gbs"], "peak": hbm, "unit": "GB/s",
                            "frac": quant["gbs"] / hbm, "traffic": None,
-                           "kernel": "k_amax + k_quantize (mq_tensor_scale + mq_nvfp4_quantize)",
+                           "kernel": "k_amax + k_quantize_tiles (mq_tensor_scale + mq_nvfp4_quantize)",
                            "bytes_per_element": 4.5625, "peak_source": f"{peaks_src}: hbm_gbs"},
         "gpu_launches": 8 * args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
         "prefill_sequence": sequence,
+        "decode_gemm": decode,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
@@ -419,6 +421,56 @@ def _prefill_sequence(args, device):
     return out
 
 
+def _decode_figure(device):
+    """Decode-shaped GEMMs (M tokens, the split-K weight-streaming kernel
+    mq_nvfp4_gemm takes for M <= 64): the four Qwen3-8B-shaped projections of
+    8 layers (weights rotate, ~0.8 GB > L2), pre-quantized operands, one CUDA
+    graph per M; weight bytes (codes + scales) per second against HBM."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    layers = 8
+    projs = inputs.QWEN3_8B_PROJECTIONS
+    weights = [[mq.quantize(inputs.weight_bf16(p.N, p.K, seed=3000 + 16 * l + i, device="cuda"))
+                for i, p in enumerate(projs)] for l in range(layers)]
+    wbytes = sum(mq.mq_nvfp4_codes_bytes(p.N, p.K) + mq.mq_nvfp4_scales_bytes(p.N, p.K) for p in projs)
+    ws = mq.workspace(mq.mq_workspace_bytes(), device)
+    out = {"workload": "qwen3-8b projections (qkv, o, gate_up, down), 8 layers of weights in rotation, one CUDA graph",
+           "weight_bytes_per_layer": wbytes}
+    for M in (1, 16, 64):
+        xs = [mq.quantize(inputs.activation_bf16(M, p.K, seed=M + i, outlier_channels=inputs.outlier_count(p.K),
+                                                 device="cuda")) for i, p in enumerate(projs)]
+        ys = [torch.empty(M, p.N, dtype=torch.bfloat16, device=device) for p in projs]
+
+        def run(stream=None):
+            for l in range(layers):
+                for i, p in enumerate(projs):
+                    q = weights[l][i]
+                    mq.mq_nvfp4_gemm(xs[i].codes, xs[i].scales, xs[i].alpha, q.codes, q.scales, q.alpha, M, p.N,
+                                     p.K, ys[i], ws, stream)
+        run()
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream(device=device)
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                run(s)
+        torch.cuda.current_stream().wait_stream(s)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / (5 * layers) * 1e3
+        out[f"M{M}"] = {"us_per_layer": us, "weight_gbs": wbytes / us / 1e3,
+                        "tflops": 2.0 * M * sum(p.N * p.K for p in projs) / us / 1e6}
+        del g
+    assert mq.mq_read_status(ws) == mq.MQ_OK
+    return out
+
+
 def _e2e(args, work, device, stream):
     """Pinned host X -> device, mq_linear_w4a4, device -> pinned host Y, per step."""
     from nvfp4_w4a4_quantized_03_b200 import mq
@@ -458,7 +510,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sequence", action="store_true",
-                    help="skip the 36-layer x 131072-token prefill-sequence figure")
+                    help="skip the 36-layer x 131072-token prefill-sequence and the decode figures")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world, rank, local = _dist()

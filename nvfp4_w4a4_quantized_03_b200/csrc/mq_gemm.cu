@@ -720,6 +720,10 @@ static bool make_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_fp4_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+    return make_code_map(map, codes, rows, K, box_rows, 128);
+}
+
 bool make_bf16_tile_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
@@ -865,6 +869,13 @@ int64_t fused_flag_count(int64_t M, int64_t K) {
 // MQ_GEMM_BK=128|256 force a variant (the tests check every variant on the
 // same shapes); the fused linear always runs with 256-element K stages.
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+    // few rows of A (decode-shaped): the weight-streaming split-K form,
+    // unless MQ_GEMM_DECODE=0 or a variant is forced
+    const char* dv = getenv("MQ_GEMM_DECODE");
+    if (!(dv && dv[0] == '0') && !getenv("MQ_GEMM_FORM") && !a.x && a.M <= 64) {
+        const cudaError_t e = launch_gemm_decode(a, num_sms, stream);
+        if (e != cudaErrorNotSupported) return e;
+    }
     const int form = env_choice("MQ_GEMM_FORM", 1, 2, a.M > gemm::BM ? 2 : 1);
     if (a.x) return form == 2 ? launch_form<2, 256, true>(a, num_sms, stream)
                               : launch_form<1, 256, true>(a, num_sms, stream);

@@ -27,6 +27,10 @@ __host__ __device__ inline int64_t padded_rows(int64_t rows) { return (rows + 12
 // boxes in the 128-byte swizzle (rows past the end read as zero).
 bool make_bf16_tile_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K, int box_rows);
 
+// Tensor map of packed E2M1 codes [rows, K/2 bytes] for TMA loads of
+// box_rows x 128-byte boxes (256 K-elements) in the 128-byte swizzle.
+bool make_fp4_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);
+
 // Launchers (enqueue on `stream`, no synchronisation).
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
                         int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0);
@@ -60,5 +64,10 @@ struct GemmArgs {
 // Readiness flags of the fused linear: one int per (128-row block, K stage).
 int64_t fused_flag_count(int64_t M, int64_t K);
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
+// Small-M form of the block-scaled GEMM (decode-shaped, M <= 64): W as the
+// MMA's 128-row operand, split-K over a cluster, partials summed through
+// distributed shared memory.  Returns cudaErrorNotSupported for shapes it
+// does not take.
+cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace mq
