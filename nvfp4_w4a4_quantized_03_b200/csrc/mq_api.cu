@@ -58,6 +58,23 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA; 
 
 }  // namespace
 
+namespace mq {
+bool pdl_enabled() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("MQ_PDL");
+        v = (e && e[0] == '0') ? 0 : 1;
+    }
+    return v == 1;
+}
+void set_pdl_attr(cudaLaunchAttribute* attr, int* nattr) {
+    if (!pdl_enabled()) return;
+    attr[*nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[*nattr].val.programmaticStreamSerializationAllowed = 1;
+    ++*nattr;
+}
+}  // namespace mq
+
 extern "C" {
 
 const char* mq_status_string(int status) {

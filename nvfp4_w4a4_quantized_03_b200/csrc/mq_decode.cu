@@ -115,6 +115,8 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = s->tmem_base;
     const volatile int* abort_flag = &s->abort_flag;
+    pdl_launch_dependents();     // set-up of the next grid may overlap this one
+    pdl_wait();                  // the grids before this one are done
     auto raise = [&]() {
         *(volatile int*)&s->abort_flag = 1;
         if (p.status) atomicExch(p.status, -7 /* MQ_ERR_TIMEOUT */);
@@ -289,7 +291,8 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stre
     }
     p.split = split;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int nattr = 1;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = split;
     attr[0].val.clusterDim.y = 1;
@@ -298,8 +301,9 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stre
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = stream;
+    set_pdl_attr(attr, &nattr);
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = nattr;
     return cudaLaunchKernelEx(&cfg, k_gemm_decode, mw, mx, p);
 }
 

@@ -239,6 +239,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t tmem = s->tmem_base;
     const volatile int* abort_flag = &s->abort_flag;
+    // the next grid may start its set-up; this one touches global memory only
+    // once the grids before it are done
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -826,7 +830,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.flags = a.flags;
     const int units = std::min(p.tiles, fs.max_units);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     int nattr = 0;
     if (PAIR == 2) {
         attr[nattr].id = cudaLaunchAttributeClusterDimension;
@@ -841,6 +845,8 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
         attr[nattr].id = cudaLaunchAttributeCooperative;
         attr[nattr].val.cooperative = 1;
         ++nattr;
+    } else {
+        set_pdl_attr(attr, &nattr);
     }
     cfg.gridDim = dim3(PAIR * units);
     cfg.blockDim = dim3(THREADS);

@@ -31,6 +31,12 @@ bool make_bf16_tile_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K
 // box_rows x 128-byte boxes (256 K-elements) in the 128-byte swizzle.
 bool make_fp4_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);
 
+// Programmatic dependent launch: each kernel lets the next grid on the
+// stream launch early and waits (griddepcontrol.wait) before its first access
+// to global memory.  Launches carry the attribute unless MQ_PDL=0.
+bool pdl_enabled();
+void set_pdl_attr(cudaLaunchAttribute* attr, int* nattr);
+
 // Launchers (enqueue on `stream`, no synchronisation).
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
                         int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0);

@@ -34,6 +34,8 @@ constexpr int AMAX_THREADS = 512;
 __global__ void __launch_bounds__(AMAX_THREADS)
 k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ tail, int ntail,
        uint32_t* __restrict__ ws, float* __restrict__ alpha_out, int* __restrict__ clear, int nclear) {
+    pdl_launch_dependents();
+    pdl_wait();
     uint32_t m = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -151,6 +153,8 @@ k_quantize_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t
         prefetch_tmap(&xmap);
     }
     __syncthreads();
+    pdl_launch_dependents();
+    pdl_wait();
     auto issue = [&](int64_t t, int st) {
         mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
         tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
@@ -202,6 +206,8 @@ k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows,
     __shared__ int ok_shared;
     __shared__ float alpha_shared;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    pdl_launch_dependents();
+    pdl_wait();
     const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(&ws[WS_GENERATION]);
     const int64_t kgroups = K / 64;
     const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
@@ -447,9 +453,17 @@ cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float*
     const uint16_t* tail = reinterpret_cast<const uint16_t*>(x) + nvec * 8;
     int64_t want = (nvec + AMAX_THREADS * 8 - 1) / (AMAX_THREADS * 8);
     int blocks = (int)std::min<int64_t>(std::max<int64_t>(want, 1), (int64_t)num_sms * 4);
-    k_amax<<<blocks, AMAX_THREADS, 0, stream>>>(reinterpret_cast<const uint4*>(x), nvec, tail, ntail,
-                                               ws_words, alpha_out, clear, nclear);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    int nattr = 0;
+    set_pdl_attr(attr, &nattr);
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(AMAX_THREADS);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = nattr;
+    return cudaLaunchKernelEx(&cfg, k_amax, reinterpret_cast<const uint4*>(x), nvec, tail, ntail, ws_words,
+                              alpha_out, clear, nclear);
 }
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
@@ -459,21 +473,30 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     CUtensorMap xmap;
     if (!(tv && tv[0] == '0') && make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) {
         static int sms[64] = {};
-        static bool attr[64] = {};
+        static bool attr_set[64] = {};
         int dev = 0;
         cudaGetDevice(&dev);
         const int d = dev < 64 ? dev : 63;
-        if (!attr[d]) {
+        if (!attr_set[d]) {
             cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
             cudaError_t e = cudaFuncSetAttribute(k_quantize_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
             if (e != cudaSuccess) return e;
-            attr[d] = true;
+            attr_set[d] = true;
         }
         const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, 2 * (int64_t)sms[d]));
-        k_quantize_tiles<<<grid, QT_THREADS, QT_SMEM, stream>>>(xmap, rows, prows, K, alpha,
-                                                                reinterpret_cast<uint4*>(codes), scales);
-        return cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        int nattr = 0;
+        set_pdl_attr(attr, &nattr);
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(QT_THREADS);
+        cfg.dynamicSmemBytes = QT_SMEM;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = nattr;
+        return cudaLaunchKernelEx(&cfg, k_quantize_tiles, xmap, rows, prows, K, alpha, reinterpret_cast<uint4*>(codes),
+                                  scales);
     }
     const int64_t threads = prows * (K / 64);
     const int64_t blocks = (threads + QUANT_THREADS - 1) / QUANT_THREADS;
