@@ -97,6 +97,27 @@ size_t mq_linear_w4a4_workspace_bytes(int64_t M, int64_t K);
 int mq_tensor_scale(const void *x, int64_t numel, float *alpha, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * max |x| of a bf16 tensor, as fp32 (exact: the largest magnitude of bf16
+ * values), for callers that shard a tensor's rows across devices: the
+ * tensor-level scale of the whole tensor ("张量级尺度", section NVFP4 微缩放量化
+ * of the paper.rainbus.top digest) is alpha_x = fl32(max over shards / 2688),
+ * so the shards' amax values are reduced (max, e.g. an NCCL all-reduce of
+ * these 4 bytes) and turned into alpha with mq_alpha_from_amax; quantizing
+ * every shard with that alpha gives the codes and scales of the unsharded
+ * tensor, row for row.
+ *   x      : device, numel bf16 values (16-byte aligned)
+ *   amax   : device, 1 float, written
+ *   ws     : as for mq_tensor_scale
+ */
+int mq_tensor_amax(const void *x, int64_t numel, float *amax, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * alpha_x = fl32(amax / 2688), or 1 if amax = 0 (the tensor-level scale of
+ * mq_tensor_scale, from a given amax).  amax and alpha: device, 1 float each.
+ */
+int mq_alpha_from_amax(const float *amax, float *alpha, void *stream);
+
+/*
  * NVFP4 quantization of a bf16 [rows, K] tensor with a given alpha_x
  * (block scale sigma_b and element codes q_i as above; section 方法步骤详情,
  * step (3); section Method, item 1).

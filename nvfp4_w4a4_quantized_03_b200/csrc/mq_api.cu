@@ -124,6 +124,26 @@ int mq_tensor_scale(const void* x, int64_t numel, float* alpha, void* ws, size_t
                                        static_cast<cudaStream_t>(stream)));
 }
 
+int mq_tensor_amax(const void* x, int64_t numel, float* amax, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !amax || numel <= 0) return MQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < mq::WS_HEADER_BYTES) return MQ_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return MQ_ERR_ALIGN;
+    int sms = 0;
+    int st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_amax(x, numel, static_cast<uint32_t*>(ws), amax, sms,
+                                       static_cast<cudaStream_t>(stream), nullptr, 0, 1));
+}
+
+int mq_alpha_from_amax(const float* amax, float* alpha, void* stream) {
+    if (!amax || !alpha) return MQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(amax) & 3u) || (reinterpret_cast<uintptr_t>(alpha) & 3u)) return MQ_ERR_ALIGN;
+    int sms = 0;
+    int st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    return cuda_status(mq::launch_alpha_from_amax(amax, alpha, static_cast<cudaStream_t>(stream)));
+}
+
 int mq_nvfp4_quantize(const void* x, int64_t rows, int64_t K, const float* alpha, uint8_t* codes,
                       uint8_t* scales, void* stream) {
     if (!x || !alpha || !codes || !scales) return MQ_ERR_INVALID_ARG;

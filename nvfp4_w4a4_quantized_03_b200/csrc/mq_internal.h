@@ -39,7 +39,8 @@ void set_pdl_attr(cudaLaunchAttribute* attr, int* nattr);
 
 // Launchers (enqueue on `stream`, no synchronisation).
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
-                        int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0);
+                        int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0, int raw_amax = 0);
+cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t stream);
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream);
 // alpha_x and the NVFP4 codes/scales of x in one cooperative launch (amax

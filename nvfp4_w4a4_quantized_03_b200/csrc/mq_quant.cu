@@ -28,12 +28,13 @@ namespace mq {
 constexpr int AMAX_THREADS = 512;
 
 // One pass over x (16-byte vectors); every block folds its max into ws with
-// one atomic, and the last block to finish turns it into alpha and resets
-// the two counters to zero.  `clear` (may be null) is zero-filled on the way:
-// the fused linear's readiness flags for this call.
+// one atomic, and the last block to finish turns it into alpha (or, with
+// raw_amax, writes max |x| itself) and resets the two counters to zero.
+// `clear` (may be null) is zero-filled on the way: the fused linear's
+// readiness flags for this call.
 __global__ void __launch_bounds__(AMAX_THREADS)
 k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ tail, int ntail,
-       uint32_t* __restrict__ ws, float* __restrict__ alpha_out, int* __restrict__ clear, int nclear) {
+       uint32_t* __restrict__ ws, float* __restrict__ alpha_out, int* __restrict__ clear, int nclear, int raw_amax) {
     pdl_launch_dependents();
     pdl_wait();
     uint32_t m = 0;
@@ -73,8 +74,7 @@ k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ t
         uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
         atomicExch(&ws[WS_TICKET], 0u);
         float amax = __uint_as_float(bits << 16);
-        float alpha = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-        *alpha_out = alpha;
+        *alpha_out = raw_amax ? amax : ((amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f));
     }
 }
 
@@ -447,7 +447,7 @@ cudaError_t launch_quantize_onepass(const void* x, int64_t rows, int64_t K, uint
 }
 
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
-                        int num_sms, cudaStream_t stream, int* clear, int nclear) {
+                        int num_sms, cudaStream_t stream, int* clear, int nclear, int raw_amax) {
     const int64_t nvec = numel / 8;
     const int ntail = (int)(numel - nvec * 8);
     const uint16_t* tail = reinterpret_cast<const uint16_t*>(x) + nvec * 8;
@@ -463,7 +463,28 @@ cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float*
     cfg.attrs = attr;
     cfg.numAttrs = nattr;
     return cudaLaunchKernelEx(&cfg, k_amax, reinterpret_cast<const uint4*>(x), nvec, tail, ntail, ws_words,
-                              alpha_out, clear, nclear);
+                              alpha_out, clear, nclear, raw_amax);
+}
+
+// alpha_x = fl32(amax / 2688), or 1 for amax = 0, from a device amax (one thread).
+__global__ void k_alpha_from_amax(const float* __restrict__ amax, float* __restrict__ alpha) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const float a = *amax;
+    *alpha = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
+}
+
+cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    int nattr = 0;
+    set_pdl_attr(attr, &nattr);
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(1);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = nattr;
+    return cudaLaunchKernelEx(&cfg, k_alpha_from_amax, amax, alpha);
 }
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,

@@ -46,12 +46,14 @@ def lib() -> ctypes.CDLL:
         L.mq_workspace_bytes.argtypes = []
         L.mq_workspace_bytes.restype = sz
         L.mq_tensor_scale.argtypes = [vp, i64, vp, vp, sz, vp]
+        L.mq_tensor_amax.argtypes = [vp, i64, vp, vp, sz, vp]
+        L.mq_alpha_from_amax.argtypes = [vp, vp, vp]
         L.mq_nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.mq_nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
         L.mq_linear_w4a4.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp, sz, vp]
         L.mq_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
-        for name in ("mq_tensor_scale", "mq_nvfp4_quantize", "mq_nvfp4_gemm", "mq_linear_w4a4",
-                     "mq_read_status"):
+        for name in ("mq_tensor_scale", "mq_tensor_amax", "mq_alpha_from_amax", "mq_nvfp4_quantize",
+                     "mq_nvfp4_gemm", "mq_linear_w4a4", "mq_read_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -102,6 +104,17 @@ def mq_tensor_scale(x: torch.Tensor, alpha: torch.Tensor, ws: torch.Tensor, stre
     assert x.dtype == torch.bfloat16 and alpha.dtype == torch.float32
     _check(lib().mq_tensor_scale(_ptr(x), x.numel(), _ptr(alpha), _ptr(ws), ws.numel() * ws.element_size(),
                                  _stream(stream)), "mq_tensor_scale")
+
+
+def mq_tensor_amax(x: torch.Tensor, amax: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    assert x.dtype == torch.bfloat16 and amax.dtype == torch.float32
+    _check(lib().mq_tensor_amax(_ptr(x), x.numel(), _ptr(amax), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)), "mq_tensor_amax")
+
+
+def mq_alpha_from_amax(amax: torch.Tensor, alpha: torch.Tensor, stream=None) -> None:
+    assert amax.dtype == torch.float32 and alpha.dtype == torch.float32
+    _check(lib().mq_alpha_from_amax(_ptr(amax), _ptr(alpha), _stream(stream)), "mq_alpha_from_amax")
 
 
 def mq_nvfp4_quantize(x: torch.Tensor, alpha: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,

@@ -65,6 +65,11 @@ def test_host_validation_without_gpu(libmq):
     assert libmq.mq_nvfp4_quantize(None, 1, 64, p16, p16, p16, None) == -1        # null
     assert libmq.mq_nvfp4_quantize(vp(4097), 1, 64, p16, p16, p16, None) == -3    # misaligned
     assert libmq.mq_tensor_scale(p16, 64, p16, p16, 16, None) == -5                # workspace too small
+    assert libmq.mq_tensor_amax(p16, 64, p16, p16, 16, None) == -5                 # workspace too small
+    assert libmq.mq_tensor_amax(None, 64, p16, p16, 256, None) == -1               # null
+    assert libmq.mq_tensor_amax(vp(4097), 64, p16, p16, 256, None) == -3           # misaligned
+    assert libmq.mq_alpha_from_amax(None, p16, None) == -1                         # null
+    assert libmq.mq_alpha_from_amax(vp(4097), p16, None) == -3                     # misaligned
     assert libmq.mq_linear_w4a4(p16, 128, 1024, p16, p16, p16, 256, p16, p16, 1024, None) == -5
     assert libmq.mq_nvfp4_gemm(p16, p16, p16, p16, p16, p16, 1, 1, 96, p16, None, 0, None) == -2
     assert libmq.mq_status_string(-7) == b"MQ_ERR_TIMEOUT"
