@@ -134,6 +134,7 @@ struct Params {
     int hints;               // bit 1: evict-first stores of Y (register path); bit 2: same for the TMA stores
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
     int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
+    int sfb_tma;             // B's two scale slices of a stage arrive as one TMA box (tmap_sfb is valid)
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
     uint8_t* x_codes;        // fused linear: where A's codes are written
     uint8_t* x_scales;       // fused linear: where A's scales are written
@@ -183,7 +184,7 @@ __device__ __forceinline__ void commit_to_all(uint64_t* bar) {
 template <int PAIR, int BK, bool QUANT>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-       const __grid_constant__ CUtensorMap tmap_y, Params p) {
+       const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfb, Params p) {
     using C = Cfg<PAIR, BK>;
     constexpr int NKB = C::NKB;
     constexpr int A_BYTES = C::A_BYTES;
@@ -223,6 +224,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
         if (C::TMA_STORE && p.y_tma) prefetch_tmap(&tmap_y);
+        if (p.sfb_tma) prefetch_tmap(&tmap_sfb);
     }
     if (warp == 1) {
         if (PAIR == 2) {
@@ -286,11 +288,19 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             tma_load_2d(stage_b(st), &tmap_b, &s->ready[st], kt * C::ROW_BYTES, brow);
                             if (!QUANT) tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
                         }
-                        mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
-                        for (int rt = 0; rt < 2; ++rt) {
-                            const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
-                            bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
-                                      p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                        if (p.sfb_tma) {
+                            // B's two 128-row scale slices in one box (rows
+                            // nb*2, nb*2+1 of the [row tile][k atom] array);
+                            // the box always lands whole, zero past the ends
+                            mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + sf_bytes);
+                            tma_load_2d(stage_sfb(st), &tmap_sfb, &s->sf_full[st], (int)(ka * 64), nb * 2);
+                        } else {
+                            mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
+                            for (int rt = 0; rt < 2; ++rt) {
+                                const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
+                                bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
+                                          p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                            }
                         }
                         if (QUANT && arow / 128 < p.a_row_tiles) {
                             // A's block (arow, kt) is written by quantizer warps (of any CTA)
@@ -740,6 +750,22 @@ bool make_bf16_tile_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The block scales of a [rows, K] operand as a 2-D array of 64-bit words:
+// [row tile][k atom x 64 words] (one 512-byte atom per 128 rows x 64 K);
+// a box is `box_rows` row tiles x `atoms` atoms, unswizzled.
+static bool make_scale_map(CUtensorMap* map, const uint8_t* scales, int64_t row_tiles, int64_t katoms,
+                           int box_rows, int atoms) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || (reinterpret_cast<uintptr_t>(scales) & 15u)) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(katoms * 64), (cuuint64_t)row_tiles};
+    cuuint64_t strides[1] = {(cuuint64_t)(katoms * 512)};
+    cuuint32_t box[2] = {(cuuint32_t)(atoms * 64), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor [M, N] for the epilogue's TMA stores: 32-row x 64-column
 // boxes in the 128-byte swizzle.  Needs N % 8 == 0 (16-byte row pitch).
 static bool make_y_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
@@ -793,12 +819,15 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
         }
         fs.attr_set = true;
     }
-    CUtensorMap ma, mb, my;
+    CUtensorMap ma, mb, my, msfb;
     if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM, C::ROW_BYTES) ||
         !make_code_map(&mb, a.b_codes, a.N, a.K, C::B_ROWS, C::ROW_BYTES))
         return cudaErrorInvalidValue;
     memset(&my, 0, sizeof(my));
     const bool y_tma = C::TMA_STORE && env_int("MQ_GEMM_YTMA", 0, 1, 1) && make_y_map(&my, a.y, a.M, a.N);
+    memset(&msfb, 0, sizeof(msfb));
+    const bool sfb_tma = env_int("MQ_GEMM_SFB_TMA", 0, 1, 1) &&
+                         make_scale_map(&msfb, a.b_scales, padded_rows(a.N) / 128, scale_atom_cols(a.K), 2, C::NKB);
     Params p{};
     p.a_scales = a.a_scales;
     p.b_scales = a.b_scales;
@@ -820,6 +849,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
     p.y_tma = y_tma ? 1 : 0;
+    p.sfb_tma = sfb_tma ? 1 : 0;
     p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
     p.hints = env_int("MQ_GEMM_HINTS", 0, 7, 0);
     p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
@@ -854,7 +884,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = nattr;
-    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, my, p);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, my, msfb, p);
 }
 
 int env_choice(const char* name, int a, int b, int dflt) {
