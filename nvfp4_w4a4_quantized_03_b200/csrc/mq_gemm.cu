@@ -135,6 +135,7 @@ struct Params {
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
     int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
     int sfb_tma;             // B's two scale slices of a stage arrive as one TMA box (tmap_sfb is valid)
+    int sfa_tma;             // A's scale slice of a stage arrives as a TMA box (tmap_sfa is valid)
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
     uint8_t* x_codes;        // fused linear: where A's codes are written
     uint8_t* x_scales;       // fused linear: where A's scales are written
@@ -184,7 +185,8 @@ __device__ __forceinline__ void commit_to_all(uint64_t* bar) {
 template <int PAIR, int BK, bool QUANT>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-       const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfb, Params p) {
+       const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfb,
+       const __grid_constant__ CUtensorMap tmap_sfa, Params p) {
     using C = Cfg<PAIR, BK>;
     constexpr int NKB = C::NKB;
     constexpr int A_BYTES = C::A_BYTES;
@@ -225,6 +227,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         prefetch_tmap(&tmap_b);
         if (C::TMA_STORE && p.y_tma) prefetch_tmap(&tmap_y);
         if (p.sfb_tma) prefetch_tmap(&tmap_sfb);
+        if (p.sfa_tma) prefetch_tmap(&tmap_sfa);
     }
     if (warp == 1) {
         if (PAIR == 2) {
@@ -292,10 +295,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             // B's two 128-row scale slices in one box (rows
                             // nb*2, nb*2+1 of the [row tile][k atom] array);
                             // the box always lands whole, zero past the ends
-                            mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + sf_bytes);
+                            mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + (p.sfa_tma ? SFB_BYTES / 2 : sf_bytes));
                             tma_load_2d(stage_sfb(st), &tmap_sfb, &s->sf_full[st], (int)(ka * 64), nb * 2);
                         } else {
-                            mbar_arrive_expect_tx(&s->sf_full[st], 3 * sf_bytes);
+                            mbar_arrive_expect_tx(&s->sf_full[st], 2 * sf_bytes + (p.sfa_tma ? SFB_BYTES / 2 : sf_bytes));
                             for (int rt = 0; rt < 2; ++rt) {
                                 const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
                                 bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
@@ -313,7 +316,10 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             }
                             fence_proxy_async_global();
                         }
-                        bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                        if (p.sfa_tma)
+                            tma_load_2d(stage_sfa(st), &tmap_sfa, &s->sf_full[st], (int)(ka * 64), (int)at);
+                        else
+                            bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
                         if (QUANT) {
                             if (PAIR == 2) tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
                             else tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
@@ -819,7 +825,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
         }
         fs.attr_set = true;
     }
-    CUtensorMap ma, mb, my, msfb;
+    CUtensorMap ma, mb, my, msfb, msfa;
     if (!make_code_map(&ma, a.a_codes, a.M, a.K, BM, C::ROW_BYTES) ||
         !make_code_map(&mb, a.b_codes, a.N, a.K, C::B_ROWS, C::ROW_BYTES))
         return cudaErrorInvalidValue;
@@ -828,6 +834,9 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     memset(&msfb, 0, sizeof(msfb));
     const bool sfb_tma = env_int("MQ_GEMM_SFB_TMA", 0, 1, 1) &&
                          make_scale_map(&msfb, a.b_scales, padded_rows(a.N) / 128, scale_atom_cols(a.K), 2, C::NKB);
+    memset(&msfa, 0, sizeof(msfa));
+    const bool sfa_tma = env_int("MQ_GEMM_SFA_TMA", 0, 1, 1) &&
+                         make_scale_map(&msfa, a.a_scales, padded_rows(a.M) / 128, scale_atom_cols(a.K), 1, C::NKB);
     Params p{};
     p.a_scales = a.a_scales;
     p.b_scales = a.b_scales;
@@ -850,6 +859,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.fault_skip_first_load = a.fault_skip_first_load;
     p.y_tma = y_tma ? 1 : 0;
     p.sfb_tma = sfb_tma ? 1 : 0;
+    p.sfa_tma = sfa_tma ? 1 : 0;
     p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
     p.hints = env_int("MQ_GEMM_HINTS", 0, 7, 0);
     p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
@@ -884,7 +894,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = nattr;
-    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, my, msfb, p);
+    return cudaLaunchKernelEx(&cfg, kernel, ma, mb, my, msfb, msfa, p);
 }
 
 int env_choice(const char* name, int a, int b, int dflt) {
