@@ -80,6 +80,14 @@ def _L():
         lib.oracle_scale_bytes.restype = i64
         lib.oracle_scales_to_stored.argtypes = [u8p, i64, i64, u8p]
         lib.oracle_scales_from_stored.argtypes = [u8p, i64, i64, u8p]
+        lib.oracle_exp_f32.argtypes = [ctypes.c_float]
+        lib.oracle_exp_f32.restype = ctypes.c_float
+        lib.oracle_silu_f32.argtypes = [ctypes.c_float]
+        lib.oracle_silu_f32.restype = ctypes.c_float
+        lib.oracle_swiglu_bf16.argtypes = [ctypes.c_uint16, ctypes.c_uint16]
+        lib.oracle_swiglu_bf16.restype = ctypes.c_uint16
+        lib.oracle_swiglu_array.argtypes = [u16p, u16p, i64, u16p]
+        lib.oracle_swiglu_array.restype = None
         _lib = lib
     return _lib
 
@@ -228,3 +236,60 @@ def unpack_codes(codes: np.ndarray) -> np.ndarray:
     out[..., 0::2] = codes & 15
     out[..., 1::2] = codes >> 4
     return out
+
+
+# -- the MLP: gate/up linear, SwiGLU, down linear ---------------------------
+
+def exp_f32(x: float) -> float:
+    """The binary32 exponential of the SwiGLU (Cody-Waite reduction, degree-7 Taylor)."""
+    return float(_L().oracle_exp_f32(float(x)))
+
+
+def silu_f32(g: float) -> float:
+    return float(_L().oracle_silu_f32(float(g)))
+
+
+def swiglu_bf16(g, u) -> np.ndarray:
+    """h = bf16(fl32(silu(g) * u)) elementwise on bf16 bit patterns."""
+    gb = np.ascontiguousarray(_bits(g))
+    ub = np.ascontiguousarray(_bits(u))
+    assert gb.shape == ub.shape
+    out = np.empty(gb.shape, np.uint16)
+    _L().oracle_swiglu_array(_p(gb, ctypes.c_uint16), _p(ub, ctypes.c_uint16), gb.size,
+                             _p(out, ctypes.c_uint16))
+    return out
+
+
+def gate_up_swiglu(x_codes, x_scales, alpha_x, wgu_codes, wgu_scales, alpha_gu, inter: int):
+    """H of the MLP from quantized operands: the gate/up product of xhat with
+    the [2 * inter, K] weight (gate rows first, then up rows), rounded to bf16
+    as the linear writes it, then SwiGLU.  Returns (h bits [M, inter], G, U)."""
+    y64 = gemm_f64(dequantize(x_codes, x_scales, alpha_x), dequantize(wgu_codes, wgu_scales, alpha_gu))
+    g = bf16_rne_array(y64[:, :inter])
+    u = bf16_rne_array(y64[:, inter:])
+    return swiglu_bf16(g, u), g, u
+
+
+def mlp_w4a4(x, wgu, wd, wgu_quant=None, wd_quant=None):
+    """End-to-end reference of the W4A4 MLP: the gate/up linear (A1-A6),
+    SwiGLU (R9, R10), the down linear on H quantized with its own alpha (R11).
+    ``wgu`` is [2 * inter, K] with the gate rows first."""
+    inter = (wgu_quant[1].shape[0] if wgu_quant is not None else _bits(wgu).shape[0]) // 2
+    ax = tensor_scale(x)
+    xc, xs = quantize(x, ax)
+    if wgu_quant is None:
+        agu = tensor_scale(wgu)
+        gc, gs = quantize(wgu, agu)
+    else:
+        agu, gc, gs = wgu_quant
+    if wd_quant is None:
+        ad = tensor_scale(wd)
+        dc, ds = quantize(wd, ad)
+    else:
+        ad, dc, ds = wd_quant
+    h, g, u = gate_up_swiglu(xc, xs, ax, gc, gs, agu, inter)
+    ah = tensor_scale(h)
+    hc, hs = quantize(h, ah)
+    y64 = gemm_f64(dequantize(hc, hs, ah), dequantize(dc, ds, ad))
+    return dict(alpha_x=ax, h=h, g=g, u=u, alpha_h=ah, h_codes=hc, h_scales=hs, y64=y64,
+                y_bf16=bf16_rne_array(y64))

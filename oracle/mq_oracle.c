@@ -343,3 +343,62 @@ void oracle_scales_from_stored(const uint8_t *stored, int64_t rows, int64_t K, u
         for (int64_t b = 0; b < K / 16; ++b)
             logical[r * (K / 16) + b] = stored[oracle_scale_offset(r, b, K)];
 }
+
+/* ------------------------------------------------------------------------- */
+/* SwiGLU of a gate/up product (the MLP between the two W4A4 linears)        */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * The pages quantize the MLP's linears but give no numerics for the gated
+ * activation between them (the down projection's input).  Readings:
+ *   R9   The gate/up product is first rounded to bf16 exactly as the plain
+ *        linear writes it: G = bf16(gate row products), U = bf16(up row
+ *        products).  Then h = bf16( fl32( silu(G) * U ) ).
+ *   R10  silu(g) = fl32( g / fl32(1 + e(-g)) ), where e(x) is a binary32
+ *        exponential built from Cody and Waite's range reduction
+ *        (x = k ln2 + r, ln2 split into a 16-bit head and a tail, |r| <= ln2/2)
+ *        and the Taylor polynomial of e^r to degree 7 in Horner form, times
+ *        2^k.  Every step is one IEEE binary32 operation (fmaf where written),
+ *        so the value does not depend on where it is evaluated.  e(x) = +inf
+ *        for x > 88 and 0 for x < -87 (k would leave the normal range).
+ *   R11  The down projection quantizes H with its own tensor scale:
+ *        alpha_h = fl32(max|h| / 2688) (R1), max over the whole [M, I] tensor.
+ */
+float oracle_exp_f32(float x)
+{
+    if (x > 88.0f) return INFINITY;
+    if (x < -87.0f) return 0.0f;
+    const float k = rintf(x * 0x1.715476p+0f);          /* nearest even of fl32(x log2 e) */
+    float r = fmaf(-k, 0x1.62e4p-1f, x);                /* x - k ln2 (head, 16 bits)       */
+    r = fmaf(-k, 0x1.7f7d1cp-20f, r);                   /* ... - k (ln2 - head)            */
+    float p = 0x1.a01a02p-13f;                          /* 1/7!                            */
+    p = fmaf(p, r, 0x1.6c16c2p-10f);                    /* 1/6!                            */
+    p = fmaf(p, r, 0x1.111112p-7f);                     /* 1/5!                            */
+    p = fmaf(p, r, 0x1.555556p-5f);                     /* 1/4!                            */
+    p = fmaf(p, r, 0x1.555556p-3f);                     /* 1/3!                            */
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    const uint32_t eb = (uint32_t)((int)k + 127) << 23; /* 2^k, k in [-126, 127]          */
+    float two_k;
+    memcpy(&two_k, &eb, sizeof two_k);
+    return p * two_k;
+}
+
+float oracle_silu_f32(float g)
+{
+    return g / (1.0f + oracle_exp_f32(-g));
+}
+
+/* h = bf16(fl32(silu(g) * u)) for bf16 g, u (R9, R10); binary32 -> bf16 RNE */
+uint16_t oracle_swiglu_bf16(uint16_t g, uint16_t u)
+{
+    const float h = oracle_silu_f32(oracle_bf16_to_f32(g)) * oracle_bf16_to_f32(u);
+    return oracle_bf16_rne((double)h);
+}
+
+void oracle_swiglu_array(const uint16_t *g, const uint16_t *u, int64_t n, uint16_t *h)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_swiglu_bf16(g[i], u[i]);
+}
