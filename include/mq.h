@@ -164,6 +164,55 @@ int mq_linear_w4a4(const void *x, int64_t M, int64_t K,
                    void *y, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The MLP's two W4A4 linears with the gated activation between them, for a
+ * decoder MLP whose gate and up projections are quantized as one weight
+ * (both linears NVFP4 W4A4 as in section 方法步骤详情, step (3); the pages give
+ * the activation no numerics, so its binary32 form is this library's):
+ *   G = bf16 gate product, U = bf16 up product (as mq_nvfp4_gemm writes them)
+ *   h = bf16( fl32( silu(G) * U ) ),  silu(g) = fl32( g / fl32(1 + e(-g)) )
+ * with e(x) the binary32 exponential by Cody and Waite's range reduction
+ * (ln 2 split into 0x1.62e4p-1 and 0x1.7f7d1cp-20) and the Taylor polynomial
+ * of e^r to degree 7, evaluated in Horner form with fused multiply-adds,
+ * times 2^k; e(x) = +inf for x > 88 and 0 for x < -87.  Every step is one
+ * IEEE binary32 operation, so H is fully determined by G and U.
+ *
+ * mq_nvfp4_gemm_swiglu: the gate/up GEMM with the activation in its epilogue.
+ *   a_codes/a_scales, alpha_a : A = [M, K] (activations)
+ *   b_codes/b_scales, alpha_b : B = [2 inter, K], rows [0, inter) the gate
+ *                               weight, rows [inter, 2 inter) the up weight,
+ *                               quantized as one tensor (one alpha)
+ *   inter    : intermediate size, a multiple of 128
+ *   h        : device bf16 [M, inter], written with H
+ *   h_amax   : device float, raised to max(*h_amax, max |h|) (set it to 0
+ *              before the first GEMM of a tensor; atomics, any order)
+ *   ws       : optional workspace as for mq_nvfp4_gemm (timeout status)
+ *
+ * mq_mlp_w4a4: y = (SwiGLU(x Wg^T, x Wu^T) quantized) Wd^T in one call:
+ *   x's tensor scale and NVFP4 form (as mq_linear_w4a4), the gate/up GEMM
+ *   above into a workspace H, alpha_h = fl32(max|h| / 2688) (1 if 0), H's
+ *   NVFP4 form, then the down GEMM.
+ *   x        : device bf16 [M, K]
+ *   wgu_*    : quantized [2 inter, K] gate/up weight as above
+ *   wd_*     : quantized down weight [N, inter]
+ *   y        : device bf16 [M, N], written
+ *   ws       : >= mq_mlp_w4a4_workspace_bytes(M, K, inter) bytes, 256-byte
+ *              aligned, zero-filled before first use (it is left that way);
+ *              calls sharing it must not overlap on the GPU.
+ * y equals mq_nvfp4_gemm on (mq_nvfp4_quantize with alpha_h)(H) and Wd bit for
+ * bit, with H and alpha_h as mq_nvfp4_gemm_swiglu and mq_alpha_from_amax
+ * give them.
+ */
+int mq_nvfp4_gemm_swiglu(const uint8_t *a_codes, const uint8_t *a_scales, const float *alpha_a,
+                         const uint8_t *b_codes, const uint8_t *b_scales, const float *alpha_b,
+                         int64_t M, int64_t inter, int64_t K, void *h, float *h_amax,
+                         void *ws, size_t ws_bytes, void *stream);
+size_t mq_mlp_w4a4_workspace_bytes(int64_t M, int64_t K, int64_t inter);
+int mq_mlp_w4a4(const void *x, int64_t M, int64_t K,
+                const uint8_t *wgu_codes, const uint8_t *wgu_scales, const float *alpha_gu, int64_t inter,
+                const uint8_t *wd_codes, const uint8_t *wd_scales, const float *alpha_d, int64_t N,
+                void *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * mq_linear_w4a4 for callers that cannot allocate device memory -- for
  * example a plugin inside a host application that owns all device memory and
  * hands extensions no allocator, or C code that must not call cudaMalloc

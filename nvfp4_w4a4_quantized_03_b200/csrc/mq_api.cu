@@ -235,6 +235,91 @@ int mq_linear_w4a4(const void* x, int64_t M, int64_t K, const uint8_t* w_codes, 
     return cuda_status(mq::launch_gemm(g, sms, s));
 }
 
+int mq_nvfp4_gemm_swiglu(const uint8_t* a_codes, const uint8_t* a_scales, const float* alpha_a,
+                         const uint8_t* b_codes, const uint8_t* b_scales, const float* alpha_b, int64_t M,
+                         int64_t inter, int64_t K, void* h, float* h_amax, void* ws, size_t ws_bytes, void* stream) {
+    if (!a_codes || !a_scales || !alpha_a || !b_codes || !b_scales || !alpha_b || !h || !h_amax)
+        return MQ_ERR_INVALID_ARG;
+    if (inter <= 0 || inter % 128 != 0) return MQ_ERR_SHAPE;
+    int st = check_rows_k(M, K);
+    if (st != MQ_OK) return st;
+    st = check_rows_k(2 * inter, K);
+    if (st != MQ_OK) return st;
+    if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
+        !aligned16(h) || (reinterpret_cast<uintptr_t>(h_amax) & 3u))
+        return MQ_ERR_ALIGN;
+    int* status = nullptr;
+    if (ws) {
+        if (ws_bytes < mq::WS_HEADER_BYTES) return MQ_ERR_WORKSPACE;
+        if (!aligned16(ws)) return MQ_ERR_ALIGN;
+        status = static_cast<int*>(ws) + mq::WS_STATUS;
+    }
+    int sms = 0;
+    st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    mq::GemmArgs g{a_codes, a_scales, alpha_a, b_codes, b_scales, alpha_b, h, M, 2 * inter, K,
+                   status, DEFAULT_TIMEOUT_CYCLES, 0};
+    g.swiglu_inter = inter;
+    g.h_amax = reinterpret_cast<uint32_t*>(h_amax);
+    return cuda_status(mq::launch_gemm(g, sms, static_cast<cudaStream_t>(stream)));
+}
+
+// Workspace of mq_mlp_w4a4: the linear's (header, flags, codes and scales of
+// X) | H bf16 [M, inter] | codes of H | scales of H.
+size_t mq_mlp_w4a4_workspace_bytes(int64_t M, int64_t K, int64_t inter) {
+    if (M <= 0 || K <= 0 || inter <= 0) return 0;
+    return mq_linear_w4a4_workspace_bytes(M, K) + round256((size_t)M * (size_t)inter * 2) +
+           round256(mq_nvfp4_codes_bytes(M, inter)) + round256(mq_nvfp4_scales_bytes(M, inter));
+}
+
+int mq_mlp_w4a4(const void* x, int64_t M, int64_t K, const uint8_t* wgu_codes, const uint8_t* wgu_scales,
+                const float* alpha_gu, int64_t inter, const uint8_t* wd_codes, const uint8_t* wd_scales,
+                const float* alpha_d, int64_t N, void* y, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !wgu_codes || !wgu_scales || !alpha_gu || !wd_codes || !wd_scales || !alpha_d || !y)
+        return MQ_ERR_INVALID_ARG;
+    if (inter <= 0 || inter % 128 != 0) return MQ_ERR_SHAPE;
+    int st = check_rows_k(M, K);
+    if (st != MQ_OK) return st;
+    if ((st = check_rows_k(2 * inter, K)) != MQ_OK || (st = check_rows_k(M, inter)) != MQ_OK ||
+        (st = check_rows_k(N, inter)) != MQ_OK)
+        return st;
+    if (!ws || ws_bytes < mq_mlp_w4a4_workspace_bytes(M, K, inter)) return MQ_ERR_WORKSPACE;
+    if (!aligned16(x) || !aligned256(ws) || !aligned16(wgu_codes) || !aligned16(wgu_scales) ||
+        !aligned16(wd_codes) || !aligned16(wd_scales) || !aligned16(y))
+        return MQ_ERR_ALIGN;
+    int sms = 0;
+    st = current_device_info(&sms);
+    if (st != MQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* words = static_cast<uint32_t*>(ws);
+    int* status = reinterpret_cast<int*>(words + mq::WS_STATUS);
+    float* alpha_x = reinterpret_cast<float*>(words + mq::WS_ALPHA);
+    float* h_amax = reinterpret_cast<float*>(words + mq::WS_H_AMAX);
+    float* alpha_h = reinterpret_cast<float*>(words + mq::WS_H_ALPHA);
+    uint8_t* x_codes = static_cast<uint8_t*>(ws) + mq::WS_HEADER_BYTES + linear_flags_bytes(M, K);
+    uint8_t* x_scales = x_codes + round256(mq_nvfp4_codes_bytes(M, K));
+    uint8_t* h = static_cast<uint8_t*>(ws) + mq_linear_w4a4_workspace_bytes(M, K);
+    uint8_t* h_codes = h + round256((size_t)M * (size_t)inter * 2);
+    uint8_t* h_scales = h_codes + round256(mq_nvfp4_codes_bytes(M, inter));
+    // 1. alpha_x and the NVFP4 form of X
+    cudaError_t e = mq::launch_quantize_onepass(x, M, K, words, alpha_x, x_codes, x_scales, status,
+                                                DEFAULT_TIMEOUT_CYCLES, s);
+    // 2. gate/up GEMM, SwiGLU and max|h| in its epilogue -> H
+    mq::GemmArgs gu{x_codes, x_scales, alpha_x, wgu_codes, wgu_scales, alpha_gu, h, M, 2 * inter, K,
+                    status, DEFAULT_TIMEOUT_CYCLES, 0};
+    gu.swiglu_inter = inter;
+    gu.h_amax = reinterpret_cast<uint32_t*>(h_amax);
+    if (e == cudaSuccess) e = mq::launch_gemm(gu, sms, s);
+    // 3. alpha_h (the running max is zeroed for the next call), NVFP4 form of H
+    if (e == cudaSuccess) e = mq::launch_alpha_from_amax(h_amax, alpha_h, s, words + mq::WS_H_AMAX);
+    if (e == cudaSuccess) e = mq::launch_quantize(h, M, inter, alpha_h, h_codes, h_scales, s);
+    // 4. down projection
+    mq::GemmArgs dn{h_codes, h_scales, alpha_h, wd_codes, wd_scales, alpha_d, y, M, N, inter,
+                    status, DEFAULT_TIMEOUT_CYCLES, 0};
+    if (e == cudaSuccess) e = mq::launch_gemm(dn, sms, s);
+    return cuda_status(e);
+}
+
 int mq_debug_gemm_stall(const uint8_t* a_codes, const uint8_t* a_scales, const float* alpha_a,
                         const uint8_t* b_codes, const uint8_t* b_scales, const float* alpha_b, int64_t M, int64_t N,
                         int64_t K, void* y, void* ws, size_t ws_bytes, int64_t timeout_cycles, void* stream) {

@@ -129,7 +129,7 @@ struct Params {
     int* status;
     long long timeout;
     int fault_skip_first_load;
-    int y_tma;               // Y is written by TMA stores (tmap_y is valid)
+    int y_tma;               // Y leaves through the staging boxes: 1 TMA stores (tmap_y is valid), 2 16-byte stores
     int pf_dist;             // L2 prefetch distance in stages (0: none)
     int hints;               // bit 1: evict-first stores of Y (register path); bit 2: same for the TMA stores
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
@@ -140,6 +140,8 @@ struct Params {
     uint8_t* x_codes;        // fused linear: where A's codes are written
     uint8_t* x_scales;       // fused linear: where A's scales are written
     int* flags;              // fused linear: [a_row_tiles][k_stages] slab counts
+    int inter;               // SwiGLU form: gate rows [0, inter), up rows [inter, 2 inter) of B
+    uint32_t* h_amax;        // SwiGLU form: running max of |h| (binary32 bits)
 };
 
 struct Smem {
@@ -154,6 +156,41 @@ struct Smem {
     uint32_t tmem_base;
     int abort_flag;
 };
+
+// SwiGLU of the MLP (gate/up product -> the down projection's input), on
+// the bf16 values the plain GEMM would write:
+//   h = bf16(fl32(silu(g) u)),  silu(g) = fl32(g / fl32(1 + e(-g))),
+// e(x) the binary32 exponential by Cody and Waite's range reduction
+// (x = k ln2 + r with ln2 split into a 16-bit head and a tail, |r| <= ln2/2)
+// and the Taylor polynomial of e^r to degree 7, each step one IEEE binary32
+// operation; +inf above 88, 0 below -87 (2^k stays a normal number).
+__device__ __forceinline__ float exp_cw(float x) {
+    if (x > 88.0f) return __int_as_float(0x7f800000);
+    if (x < -87.0f) return 0.0f;
+    const float k = rintf(__fmul_rn(x, 0x1.715476p+0f));
+    float r = __fmaf_rn(-k, 0x1.62e4p-1f, x);
+    r = __fmaf_rn(-k, 0x1.7f7d1cp-20f, r);
+    float e = 0x1.a01a02p-13f;
+    e = __fmaf_rn(e, r, 0x1.6c16c2p-10f);
+    e = __fmaf_rn(e, r, 0x1.111112p-7f);
+    e = __fmaf_rn(e, r, 0x1.555556p-5f);
+    e = __fmaf_rn(e, r, 0x1.555556p-3f);
+    e = __fmaf_rn(e, r, 0.5f);
+    e = __fmaf_rn(e, r, 1.0f);
+    e = __fmaf_rn(e, r, 1.0f);
+    return __fmul_rn(e, __int_as_float(((int)k + 127) << 23));
+}
+
+__device__ __forceinline__ float swiglu_f32(float g, float u) {
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, exp_cw(-g))), u);
+}
+
+// two bf16 pairs (g, u packed as bf16x2) -> h packed as bf16x2
+__device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
+    const float h_lo = swiglu_f32(__uint_as_float(g2 << 16), __uint_as_float(u2 << 16));
+    const float h_hi = swiglu_f32(__uint_as_float(g2 & 0xffff0000u), __uint_as_float(u2 & 0xffff0000u));
+    return cvt_bf16x2(h_hi, h_lo);
+}
 
 __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
     const int group = p.group_m * p.n_blocks;
@@ -182,7 +219,7 @@ __device__ __forceinline__ void commit_to_all(uint64_t* bar) {
     else mma_commit(bar);
 }
 
-template <int PAIR, int BK, bool QUANT>
+template <int PAIR, int BK, bool QUANT, bool SWIGLU>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
        const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfb,
@@ -195,6 +232,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
     constexpr uint32_t SF_COLS_PER_STAGE = C::SF_COLS_PER_STAGE;
     constexpr uint32_t SFB_OFF = C::SFB_OFF;
     static_assert(sizeof(Smem) <= BARRIER_BYTES, "barrier area");
+    static_assert(!SWIGLU || (PAIR == 2 && !QUANT && C::B_ROWS == 128), "SwiGLU form: pair tiles, gate | up halves");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_stage = base + C::STAGES * C::STAGE_BYTES;          // 1024-byte aligned
@@ -261,7 +299,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 int mb, nb;
                 tile_coords(tile, p, mb, nb);
                 const int arow = mb * C::TILE_M + (int)rank * BM;          // this CTA's A rows
-                const int brow = nb * BN + (int)rank * C::B_ROWS;          // this CTA's B rows
+                // this CTA's B rows (SwiGLU form: CTA 0 the gate rows, CTA 1 the matching up rows)
+                const int brow = SWIGLU ? (int)rank * p.inter + nb * 128 : nb * BN + (int)rank * C::B_ROWS;
                 // scale rows past the padded end feed only discarded outputs
                 const int64_t at = min(arow / 128, p.a_row_tiles - 1);
                 for (int kt = 0; kt < p.k_stages; ++kt) {
@@ -291,7 +330,11 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             tma_load_2d(stage_b(st), &tmap_b, &s->ready[st], kt * C::ROW_BYTES, brow);
                             if (!QUANT) tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
                         }
-                        if (p.sfb_tma) {
+                        if (SWIGLU) {
+                            // the gate and the up scale slices in one box of a 3-D view
+                            mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + (p.sfa_tma ? SFB_BYTES / 2 : sf_bytes));
+                            tma_load_3d(stage_sfb(st), &tmap_sfb, &s->sf_full[st], (int)(ka * 64), nb, 0);
+                        } else if (p.sfb_tma) {
                             // B's two 128-row scale slices in one box (rows
                             // nb*2, nb*2+1 of the [row tile][k atom] array);
                             // the box always lands whole, zero past the ends
@@ -335,7 +378,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             int mb2, nb2;
                             tile_coords(tile2, p, mb2, nb2);
                             const int arow2 = mb2 * C::TILE_M + (int)rank * BM;
-                            const int brow2 = nb2 * BN + (int)rank * C::B_ROWS;
+                            const int brow2 = SWIGLU ? (int)rank * p.inter + nb2 * 128 : nb2 * BN + (int)rank * C::B_ROWS;
                             tma_prefetch_2d(&tmap_b, kt2 * C::ROW_BYTES, brow2);
                             if (!QUANT) tma_prefetch_2d(&tmap_a, kt2 * C::ROW_BYTES, arow2);
                         }
@@ -559,7 +602,68 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
             const int row = mb * C::TILE_M + (int)rank * BM + quad * 32 + lane;
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
             const int colh = nb * BN + half * 128;
-            if (C::TMA_STORE && p.y_tma) {
+            if constexpr (SWIGLU) {
+                // Gate columns [64 half, 64 half + 64) of the accumulator and
+                // the up columns 128 above them, for this warp's 32 rows: G and
+                // U are rounded to bf16 as the plain GEMM would write them,
+                // TMEM goes back to the MMA thread once the four 32-column
+                // loads have landed, then h = SwiGLU(G, U) leaves as one
+                // 32 x 64 box of H [M, inter] (columns 128 nb + 64 half) and
+                // max|h| joins the tensor's running maximum.
+                uint8_t* box = epi_stage + (warp - FIRST_EPI_WARP) * C::EPI_BOX_BYTES;
+                const uint32_t box_row = smem_u32(box) + lane * 128;
+                const int row0 = mb * C::TILE_M + (int)rank * BM + quad * 32;
+                const uint32_t tg = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 64;
+                const uint32_t tu = tg + 128;
+                auto convert = [&](const uint32_t (&r)[32], uint32_t (&pk)[16]) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        pk[j] = cvt_bf16x2(__fmul_rn(__uint_as_float(r[2 * j + 1]), ab),
+                                           __fmul_rn(__uint_as_float(r[2 * j]), ab));
+                };
+                if (lane == 0) bulk_wait_group_read0();         // the previous tile's box has been read
+                __syncwarp();
+                uint32_t ra[32], rb[32], gq[2][16], uq[2][16];
+                tmem_ld_32x32b_x32(tg, ra);
+                tmem_ld_wait_regs(ra);
+                tmem_ld_32x32b_x32(tu, rb);
+                convert(ra, gq[0]);
+                tmem_ld_wait_regs(rb);
+                tmem_ld_32x32b_x32(tg + 32, ra);
+                convert(rb, uq[0]);
+                tmem_ld_wait_regs(ra);
+                tmem_ld_32x32b_x32(tu + 32, rb);
+                convert(ra, gq[1]);
+                tmem_ld_wait_regs(rb);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
+                convert(rb, uq[1]);
+                uint32_t hmax = 0;                              // max |h| as a bf16 bit pattern
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t hq[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        hq[j] = swiglu_bf16x2(gq[c][j], uq[c][j]);
+                        hmax = max(hmax, max(hq[j] & 0x7fffu, (hq[j] >> 16) & 0x7fffu));
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_shared_v4(box_row + (((c * 4 + q) ^ (lane & 7)) << 4), hq[4 * q], hq[4 * q + 1],
+                                     hq[4 * q + 2], hq[4 * q + 3]);
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                const int hcol = nb * 128 + half * 64;
+                if (lane == 0 && row0 < p.M) {
+                    tma_store_2d(&tmap_y, box, hcol, row0);
+                    bulk_commit_group();
+                }
+                // rows past M hold h = 0 (A reads as zero there)
+                hmax = __reduce_max_sync(0xffffffffu, hmax);
+                if (lane == 0 && hmax != 0) atomicMax(p.h_amax, hmax << 16);
+            } else if (C::TMA_STORE && p.y_tma) {
                 // This warp's 32 x 128 block of the accumulator leaves as two
                 // 32 x 64 bf16 boxes through the warp's staging buffer (TMA
                 // stores clip rows >= M and columns >= N).  The four 32-column
@@ -574,6 +678,23 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     st_shared_v4(box_row + ((j ^ (lane & 7)) << 4), v[0], v[1], v[2], v[3]);
                 };
                 auto issue = [&](int h) {
+                    if (p.y_tma == 2) {
+                        // the warp copies its box to Y: 8 lanes per 128-byte
+                        // box row, 4 rows per instruction (the TMA unit keeps
+                        // to the operand loads)
+                        __syncwarp();
+                        const int ch = lane & 7;
+                        const int col = colh + h * 64 + ch * 8;
+#pragma unroll
+                        for (int it = 0; it < 8; ++it) {
+                            const int rr = it * 4 + (lane >> 3);
+                            const uint4 v = ld_shared_v4(smem_u32(box) + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                            if (row0 + rr < p.M && col < p.N)
+                                *reinterpret_cast<uint4*>(p.y + (int64_t)(row0 + rr) * p.N + col) = v;
+                        }
+                        __syncwarp();
+                        return;
+                    }
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0 && row0 < p.M && colh + h * 64 < p.N) {
@@ -772,6 +893,22 @@ static bool make_scale_map(CUtensorMap* map, const uint8_t* scales, int64_t row_
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The scales of a [2 inter, K] gate/up operand as a 3-D array of 64-bit
+// words [half][row tile][k atom x 64 words]: one box (`atoms` atoms x 1 row
+// tile x 2 halves) brings a gate slice and the matching up slice.
+static bool make_gate_up_scale_map(CUtensorMap* map, const uint8_t* scales, int64_t inter, int64_t katoms,
+                                   int atoms) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || inter % 128 != 0 || (reinterpret_cast<uintptr_t>(scales) & 15u)) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)(katoms * 64), (cuuint64_t)(inter / 128), 2};
+    cuuint64_t strides[2] = {(cuuint64_t)(katoms * 512), (cuuint64_t)(inter / 128 * katoms * 512)};
+    cuuint32_t box[3] = {(cuuint32_t)(atoms * 64), 1, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<uint8_t*>(scales), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor [M, N] for the epilogue's TMA stores: 32-row x 64-column
 // boxes in the 128-byte swizzle.  Needs N % 8 == 0 (16-byte row pitch).
 static bool make_y_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
@@ -792,16 +929,16 @@ struct FormState {
     bool attr_set = false;
     int max_units = 0;      // co-resident CTAs (PAIR 1) or clusters (PAIR 2)
 };
-FormState g_form[64][3][2][2];
+FormState g_form[64][3][2][2][2];
 
-template <int PAIR, int BK, bool QUANT>
+template <int PAIR, int BK, bool QUANT, bool SWIGLU = false>
 cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     using namespace gemm;
     using C = Cfg<PAIR, BK>;
     int dev = 0;
     cudaGetDevice(&dev);
-    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][BK == 256][QUANT];
-    auto kernel = k_gemm<PAIR, BK, QUANT>;
+    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][BK == 256][QUANT][SWIGLU];
+    auto kernel = k_gemm<PAIR, BK, QUANT, SWIGLU>;
     if (!fs.attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
@@ -830,10 +967,21 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
         !make_code_map(&mb, a.b_codes, a.N, a.K, C::B_ROWS, C::ROW_BYTES))
         return cudaErrorInvalidValue;
     memset(&my, 0, sizeof(my));
-    const bool y_tma = C::TMA_STORE && env_int("MQ_GEMM_YTMA", 0, 1, 1) && make_y_map(&my, a.y, a.M, a.N);
     memset(&msfb, 0, sizeof(msfb));
-    const bool sfb_tma = env_int("MQ_GEMM_SFB_TMA", 0, 1, 1) &&
-                         make_scale_map(&msfb, a.b_scales, padded_rows(a.N) / 128, scale_atom_cols(a.K), 2, C::NKB);
+    // the SwiGLU form writes H [M, inter] (inter = N / 2) by TMA stores
+    const int64_t n_out = SWIGLU ? a.swiglu_inter : a.N;
+    const int y_mode = SWIGLU ? 1 : env_int("MQ_GEMM_YTMA", 0, 2, 1);
+    const bool y_tma = C::TMA_STORE && y_mode != 0 && make_y_map(&my, a.y, a.M, n_out);
+    bool sfb_tma;
+    if (SWIGLU) {
+        if (!y_tma || a.N != 2 * a.swiglu_inter || !a.h_amax ||
+            !make_gate_up_scale_map(&msfb, a.b_scales, a.swiglu_inter, scale_atom_cols(a.K), C::NKB))
+            return cudaErrorInvalidValue;
+        sfb_tma = true;
+    } else {
+        sfb_tma = env_int("MQ_GEMM_SFB_TMA", 0, 1, 1) &&
+                  make_scale_map(&msfb, a.b_scales, padded_rows(a.N) / 128, scale_atom_cols(a.K), 2, C::NKB);
+    }
     memset(&msfa, 0, sizeof(msfa));
     const bool sfa_tma = env_int("MQ_GEMM_SFA_TMA", 0, 1, 1) &&
                          make_scale_map(&msfa, a.a_scales, padded_rows(a.M) / 128, scale_atom_cols(a.K), 1, C::NKB);
@@ -844,10 +992,12 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.alpha_b = a.alpha_b;
     p.y = reinterpret_cast<__nv_bfloat16*>(a.y);
     p.M = (int)a.M;
-    p.N = (int)a.N;
+    p.N = (int)n_out;
     p.K = (int)a.K;
     p.m_blocks = (int)((a.M + C::TILE_M - 1) / C::TILE_M);
-    p.n_blocks = (int)((a.N + BN - 1) / BN);
+    p.n_blocks = SWIGLU ? (int)(a.swiglu_inter / 128) : (int)((a.N + BN - 1) / BN);
+    p.inter = (int)a.swiglu_inter;
+    p.h_amax = a.h_amax;
     p.tiles = p.m_blocks * p.n_blocks;
     p.kblocks = (int)(a.K / MMA_K);
     p.k_stages = (p.kblocks + C::NKB - 1) / C::NKB;
@@ -857,7 +1007,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.status = a.status;
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
-    p.y_tma = y_tma ? 1 : 0;
+    p.y_tma = y_tma ? y_mode : 0;
     p.sfb_tma = sfb_tma ? 1 : 0;
     p.sfa_tma = sfa_tma ? 1 : 0;
     p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
@@ -915,6 +1065,7 @@ int64_t fused_flag_count(int64_t M, int64_t K) {
 // MQ_GEMM_BK=128|256 force a variant (the tests check every variant on the
 // same shapes); the fused linear always runs with 256-element K stages.
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+    if (a.swiglu_inter > 0) return launch_form<2, 256, false, true>(a, num_sms, stream);
     // few rows of A (decode-shaped): the weight-streaming split-K form,
     // unless MQ_GEMM_DECODE=0 or a variant is forced
     const char* dv = getenv("MQ_GEMM_DECODE");

@@ -15,6 +15,8 @@ enum WsWord : int {
     WS_STATUS = 2,      // device-side status (0 = ok, else an mq_status code)
     WS_ALPHA = 3,       // alpha_x written by the amax pass of mq_linear_w4a4
     WS_GENERATION = 4,  // grid-barrier generation of the one-pass quantizer (only grows)
+    WS_H_AMAX = 5,      // mq_mlp_w4a4: running max of |h| (binary32 bits), zeroed once read
+    WS_H_ALPHA = 6,     // mq_mlp_w4a4: alpha_h of the down projection's input
 };
 constexpr size_t WS_HEADER_BYTES = 256;
 
@@ -40,7 +42,8 @@ void set_pdl_attr(cudaLaunchAttribute* attr, int* nattr);
 // Launchers (enqueue on `stream`, no synchronisation).
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
                         int num_sms, cudaStream_t stream, int* clear = nullptr, int nclear = 0, int raw_amax = 0);
-cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t stream);
+cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t stream,
+                                   uint32_t* reset = nullptr);
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream);
 // alpha_x and the NVFP4 codes/scales of x in one cooperative launch (amax
@@ -66,6 +69,12 @@ struct GemmArgs {
     // alpha_a, publishing each 128-row x (stage) block through `flags`.
     const void* x = nullptr;
     int* flags = nullptr;
+    // The MLP's gate/up GEMM with SwiGLU in the epilogue: B is [2 inter, K]
+    // (gate rows, then up rows; inter % 128 == 0, N = 2 inter), y receives
+    // H = SwiGLU(G, U) as bf16 [M, inter] and h_amax the running max of |h|
+    // (binary32 bits, atomically raised).
+    int64_t swiglu_inter = 0;
+    uint32_t* h_amax = nullptr;
 };
 
 // Readiness flags of the fused linear: one int per (128-row block, K stage).

@@ -467,14 +467,17 @@ cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float*
 }
 
 // alpha_x = fl32(amax / 2688), or 1 for amax = 0, from a device amax (one thread).
-__global__ void k_alpha_from_amax(const float* __restrict__ amax, float* __restrict__ alpha) {
+// alpha = fl32(amax / 2688) (1 when amax = 0); `reset`, when given, is
+// zeroed after the read (a running maximum ready for the next call).
+__global__ void k_alpha_from_amax(const float* amax, float* alpha, uint32_t* reset) {
     pdl_launch_dependents();
     pdl_wait();
     const float a = *amax;
     *alpha = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
+    if (reset) *reset = 0u;
 }
 
-cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t stream) {
+cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t stream, uint32_t* reset) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     int nattr = 0;
@@ -484,7 +487,7 @@ cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = nattr;
-    return cudaLaunchKernelEx(&cfg, k_alpha_from_amax, amax, alpha);
+    return cudaLaunchKernelEx(&cfg, k_alpha_from_amax, amax, alpha, reset);
 }
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,

@@ -52,8 +52,13 @@ def lib() -> ctypes.CDLL:
         L.mq_nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
         L.mq_linear_w4a4.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp, sz, vp]
         L.mq_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.mq_nvfp4_gemm_swiglu.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, sz, vp]
+        L.mq_mlp_w4a4_workspace_bytes.argtypes = [i64, i64, i64]
+        L.mq_mlp_w4a4_workspace_bytes.restype = sz
+        L.mq_mlp_w4a4.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, sz, vp]
         for name in ("mq_tensor_scale", "mq_tensor_amax", "mq_alpha_from_amax", "mq_nvfp4_quantize",
-                     "mq_nvfp4_gemm", "mq_linear_w4a4", "mq_read_status"):
+                     "mq_nvfp4_gemm", "mq_linear_w4a4", "mq_read_status", "mq_nvfp4_gemm_swiglu",
+                     "mq_mlp_w4a4"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -144,6 +149,28 @@ def mq_linear_w4a4(x: torch.Tensor, w_codes, w_scales, alpha_w, N: int, y: torch
                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "mq_linear_w4a4")
 
 
+def mq_nvfp4_gemm_swiglu(a_codes, a_scales, alpha_a, b_codes, b_scales, alpha_b, M: int, inter: int, K: int,
+                         h: torch.Tensor, h_amax: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> None:
+    assert h.dtype == torch.bfloat16 and h.numel() >= M * inter and h_amax.dtype == torch.float32
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().mq_nvfp4_gemm_swiglu(_ptr(a_codes), _ptr(a_scales), _ptr(alpha_a), _ptr(b_codes), _ptr(b_scales),
+                                      _ptr(alpha_b), M, inter, K, _ptr(h), _ptr(h_amax), _ptr(ws), ws_bytes,
+                                      _stream(stream)), "mq_nvfp4_gemm_swiglu")
+
+
+def mq_mlp_w4a4_workspace_bytes(M: int, K: int, inter: int) -> int:
+    return int(lib().mq_mlp_w4a4_workspace_bytes(M, K, inter))
+
+
+def mq_mlp_w4a4(x: torch.Tensor, wgu_codes, wgu_scales, alpha_gu, inter: int, wd_codes, wd_scales, alpha_d,
+                N: int, y: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and y.dtype == torch.bfloat16
+    M, K = x.shape
+    _check(lib().mq_mlp_w4a4(_ptr(x), M, K, _ptr(wgu_codes), _ptr(wgu_scales), _ptr(alpha_gu), inter,
+                             _ptr(wd_codes), _ptr(wd_scales), _ptr(alpha_d), N, _ptr(y), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "mq_mlp_w4a4")
+
+
 def mq_read_status(ws: torch.Tensor, stream=None) -> int:
     out = ctypes.c_int32(0)
     _check(lib().mq_read_status(_ptr(ws), _stream(stream), ctypes.byref(out)), "mq_read_status")
@@ -198,6 +225,44 @@ class LinearW4A4:
             out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         mq_linear_w4a4(x, self.w.codes, self.w.scales, self.w.alpha, self.N, out, self._ws, stream)
         return out
+
+
+class MLPW4A4:
+    """A decoder MLP on the FP4 prefill path: y = (SwiGLU(x Wg^T, x Wu^T)) Wd^T
+    with both linears W4A4.  The gate and up weights are quantized as one
+    [2 inter, K] tensor (gate rows first), the down weight [N, inter] on its
+    own, once at construction; x and H are quantized per call."""
+
+    def __init__(self, w_gate_up: torch.Tensor, w_down: torch.Tensor):
+        assert w_gate_up.dtype == torch.bfloat16 and w_down.dtype == torch.bfloat16
+        two_inter, self.K = w_gate_up.shape
+        self.inter = two_inter // 2
+        self.N = w_down.shape[0]
+        assert two_inter == 2 * self.inter and w_down.shape[1] == self.inter
+        self.wgu = quantize(w_gate_up.contiguous())
+        self.wd = quantize(w_down.contiguous())
+        self._ws = None
+
+    def workspace(self, M: int, device) -> torch.Tensor:
+        need = mq_mlp_w4a4_workspace_bytes(M, self.K, self.inter)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = workspace(need, device)
+        return self._ws
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        M, K = x.shape
+        assert K == self.K
+        ws = self.workspace(M, x.device)
+        if out is None:
+            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        mq_mlp_w4a4(x, self.wgu.codes, self.wgu.scales, self.wgu.alpha, self.inter, self.wd.codes, self.wd.scales,
+                    self.wd.alpha, self.N, out, ws, stream)
+        return out
+
+    def h_view(self, M: int) -> torch.Tensor:
+        """H [M, inter] as the last call left it in the workspace."""
+        off = mq_linear_w4a4_workspace_bytes(M, self.K)
+        return self._ws[off:off + M * self.inter * 2].view(torch.bfloat16).view(M, self.inter)
 
 
 # -- the allocation-free variant (library-owned scratch) ---------------------

@@ -54,6 +54,8 @@ def test_sizes(libmq):
     assert mq.mq_workspace_bytes() == 256
     # header | readiness flags (1 row tile x 4 K stages, padded to 256 B) | codes | scales
     assert mq.mq_linear_w4a4_workspace_bytes(128, 1024) == 256 + 256 + 65536 + 8192
+    # the linear's workspace | H bf16 | codes of H | scales of H
+    assert mq.mq_mlp_w4a4_workspace_bytes(128, 1024, 256) == 74240 + 65536 + 16384 + 2048
 
 
 def test_host_validation_without_gpu(libmq):
@@ -72,4 +74,14 @@ def test_host_validation_without_gpu(libmq):
     assert libmq.mq_alpha_from_amax(vp(4097), p16, None) == -3                     # misaligned
     assert libmq.mq_linear_w4a4(p16, 128, 1024, p16, p16, p16, 256, p16, p16, 1024, None) == -5
     assert libmq.mq_nvfp4_gemm(p16, p16, p16, p16, p16, p16, 1, 1, 96, p16, None, 0, None) == -2
+    # gate/up GEMM with SwiGLU: inter a multiple of 128, h_amax required and 4-byte aligned
+    assert libmq.mq_nvfp4_gemm_swiglu(p16, p16, p16, p16, p16, p16, 256, 100, 1024, p16, p16, None, 0, None) == -2
+    assert libmq.mq_nvfp4_gemm_swiglu(p16, p16, p16, p16, p16, p16, 256, 128, 1024, p16, None, None, 0, None) == -1
+    assert libmq.mq_nvfp4_gemm_swiglu(p16, p16, p16, p16, p16, p16, 256, 128, 1024, p16, vp(4098), None, 0,
+                                      None) == -3
+    assert libmq.mq_nvfp4_gemm_swiglu(p16, p16, p16, p16, p16, p16, 256, 128, 96, p16, p16, None, 0, None) == -2
+    # the MLP: workspace size, inter a multiple of 128
+    assert libmq.mq_mlp_w4a4(p16, 128, 1024, p16, p16, p16, 256, p16, p16, p16, 64, p16, p16, 1024, None) == -5
+    assert libmq.mq_mlp_w4a4(p16, 128, 1024, p16, p16, p16, 64, p16, p16, p16, 64, p16, p16, 1 << 30, None) == -2
+    assert libmq.mq_mlp_w4a4(p16, 128, 1024, None, p16, p16, 256, p16, p16, p16, 64, p16, p16, 1 << 30, None) == -1
     assert libmq.mq_status_string(-7) == b"MQ_ERR_TIMEOUT"
