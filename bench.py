@@ -282,6 +282,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
     sequence = None if args.no_sequence else _prefill_sequence(args, device)
     decode = None if args.no_sequence else _decode_figure(device)
+    mlp = None if args.no_sequence else _mlp_figure(device)
 
     peaks, peaks_src = _peaks()
     fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]        # nominal fp4 : bf16 = 9 : 2.25
@@ -316,6 +317,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
         "prefill_sequence": sequence,
         "decode_gemm": decode,
+        "mlp": mlp,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
@@ -471,6 +473,47 @@ def _decode_figure(device):
     return out
 
 
+def _mlp_figure(device):
+    """The Qwen3-8B-shaped MLP at 8192 tokens (K 4096, inter 12288, N 4096):
+    mq_mlp_w4a4 (x quantized, gate/up GEMM with SwiGLU and max|h| in its
+    epilogue, alpha_h, H quantized, down GEMM) against the two linears alone
+    (mq_linear_w4a4 on gate/up writing [M, 2 inter], then on the down
+    projection with a fixed input), which do not compute the activation."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    M, K, inter, N = TOKENS, 4096, 12288, 4096
+    x = inputs.activation_bf16(M, K, seed=4000, outlier_channels=inputs.outlier_count(K), outlier_scale=50.0,
+                               device="cuda")
+    wgu = inputs.weight_bf16(2 * inter, K, seed=4001, device="cuda")
+    wd = inputs.weight_bf16(N, inter, seed=4002, device="cuda")
+    mlp = mq.MLPW4A4(wgu, wd)
+    lin_gu, lin_d = mq.LinearW4A4(wgu), mq.LinearW4A4(wd)
+    del wgu, wd
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    y_gu = torch.empty(M, 2 * inter, dtype=torch.bfloat16, device=device)
+    mlp(x, y)
+    h = mlp.h_view(M).clone()
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms_mlp = timed(lambda: mlp(x, y))
+    ms_two = timed(lambda: (lin_gu(x, y_gu), lin_d(h, y)))
+    assert mq.mq_read_status(mlp._ws) == mq.MQ_OK
+    flops = 2.0 * M * K * 2 * inter + 2.0 * M * inter * N
+    return {"workload": "qwen3-8b MLP at 8192 tokens: x [8192, 4096], gate/up [24576, 4096], down [4096, 12288]",
+            "ms": ms_mlp, "tflops": flops / ms_mlp / 1e9,
+            "two_linears_without_activation_ms": ms_two,
+            "launches": 5, "flops": flops}
+
+
 def _e2e(args, work, device, stream):
     """Pinned host X -> device, mq_linear_w4a4, device -> pinned host Y, per step."""
     from nvfp4_w4a4_quantized_03_b200 import mq
@@ -510,7 +553,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sequence", action="store_true",
-                    help="skip the 36-layer x 131072-token prefill-sequence and the decode figures")
+                    help="skip the 36-layer x 131072-token prefill-sequence, decode and MLP figures")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world, rank, local = _dist()
