@@ -15,7 +15,9 @@ Formulas followed (NVFP4 two-level microscaling):
     sigma_b = Pi_E4M3(max_{i in b}|x_i| / (alpha_x q_max)),
     q_i = Pi_FP4(x_i / (alpha_x sigma_b(i))),  xhat_i = alpha_x sigma_b(i) q_i,
   blocks of 16 along K, round to nearest.  The readings taken where the pages
-  are silent are listed at the top of ``mq_oracle.c`` (R1..R8).
+  are silent are listed in ``mq_oracle.c`` (R1..R8 at the top, R11..R13 with
+  the SwiGLU of the MLP; R9 and R10, the block axis and one alpha per fused
+  weight, are how the inputs are laid out).
 """
 from __future__ import annotations
 
@@ -272,7 +274,7 @@ def gate_up_swiglu(x_codes, x_scales, alpha_x, wgu_codes, wgu_scales, alpha_gu, 
 
 def mlp_w4a4(x, wgu, wd, wgu_quant=None, wd_quant=None):
     """End-to-end reference of the W4A4 MLP: the gate/up linear (A1-A6),
-    SwiGLU (R9, R10), the down linear on H quantized with its own alpha (R11).
+    SwiGLU (R11, R12), the down linear on H quantized with its own alpha (R13).
     ``wgu`` is [2 * inter, K] with the gate rows first."""
     inter = (wgu_quant[1].shape[0] if wgu_quant is not None else _bits(wgu).shape[0]) // 2
     ax = tensor_scale(x)

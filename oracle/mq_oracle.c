@@ -351,17 +351,17 @@ void oracle_scales_from_stored(const uint8_t *stored, int64_t rows, int64_t K, u
 /*
  * The pages quantize the MLP's linears but give no numerics for the gated
  * activation between them (the down projection's input).  Readings:
- *   R9   The gate/up product is first rounded to bf16 exactly as the plain
+ *   R11  The gate/up product is first rounded to bf16 exactly as the plain
  *        linear writes it: G = bf16(gate row products), U = bf16(up row
  *        products).  Then h = bf16( fl32( silu(G) * U ) ).
- *   R10  silu(g) = fl32( g / fl32(1 + e(-g)) ), where e(x) is a binary32
+ *   R12  silu(g) = fl32( g / fl32(1 + e(-g)) ), where e(x) is a binary32
  *        exponential built from Cody and Waite's range reduction
  *        (x = k ln2 + r, ln2 split into a 16-bit head and a tail, |r| <= ln2/2)
  *        and the Taylor polynomial of e^r to degree 7 in Horner form, times
  *        2^k.  Every step is one IEEE binary32 operation (fmaf where written),
  *        so the value does not depend on where it is evaluated.  e(x) = +inf
  *        for x > 88 and 0 for x < -87 (k would leave the normal range).
- *   R11  The down projection quantizes H with its own tensor scale:
+ *   R13  The down projection quantizes H with its own tensor scale:
  *        alpha_h = fl32(max|h| / 2688) (R1), max over the whole [M, I] tensor.
  */
 float oracle_exp_f32(float x)
@@ -390,7 +390,7 @@ float oracle_silu_f32(float g)
     return g / (1.0f + oracle_exp_f32(-g));
 }
 
-/* h = bf16(fl32(silu(g) * u)) for bf16 g, u (R9, R10); binary32 -> bf16 RNE */
+/* h = bf16(fl32(silu(g) * u)) for bf16 g, u (R11, R12); binary32 -> bf16 RNE */
 uint16_t oracle_swiglu_bf16(uint16_t g, uint16_t u)
 {
     const float h = oracle_silu_f32(oracle_bf16_to_f32(g)) * oracle_bf16_to_f32(u);

@@ -4,7 +4,7 @@ GEMM + SwiGLU + max|h|, alpha_h, quantize H, down GEMM).
 
 Both linears are NVFP4 W4A4 ("Mix-Quant：面向智能体LLM的量化预填充与精确解码",
 section 方法步骤详情, step (3)); the gated activation between them follows the
-oracle's readings R9-R11 (bf16 G and U, binary32 SwiGLU, H quantized with its
+oracle's readings R11-R13 (bf16 G and U, binary32 SwiGLU, H quantized with its
 own tensor scale).
 
   * bit-exact: operands whose products and partial sums are exact in
@@ -64,7 +64,7 @@ def test_swiglu_gemm_bit_exact(M, inter, K):
     bad = np.argwhere(got != ref)
     assert len(bad) == 0, f"{len(bad)} mismatches, first {bad[:4].tolist()}"
     assert amax == float(np.max(np.abs(bf16_bits_to_f64(ref))))
-    # H's NVFP4 form with its own tensor scale (R11), bit for bit
+    # H's NVFP4 form with its own tensor scale (R13), bit for bit
     ah = oracle.tensor_scale(ref)
     alpha = torch.empty(1, dtype=torch.float32, device=dev())
     mq.mq_alpha_from_amax(torch.tensor([amax], dtype=torch.float32, device=dev()), alpha)

@@ -1,7 +1,7 @@
 """Pins of the oracle's SwiGLU, the activation between the MLP's gate/up and
 down W4A4 linears (the pages quantize both linears, "Mix-Quant：面向智能体LLM的
 量化预填充与精确解码", section 方法步骤详情, step (3); they give the gated
-activation no numerics, so its binary32 form is a reading: R9-R11 in the
+activation no numerics, so its binary32 form is a reading: R11-R13 in the
 oracle's source).
 
 Pins, none of which re-types the oracle's formula:
