@@ -129,7 +129,7 @@ struct Params {
     int* status;
     long long timeout;
     int fault_skip_first_load;
-    int y_tma;               // Y leaves through the staging boxes: 1 TMA stores (tmap_y is valid), 2 16-byte stores
+    int y_tma;               // Y is written by TMA stores (tmap_y is valid)
     int pf_dist;             // L2 prefetch distance in stages (0: none)
     int hints;               // bit 1: evict-first stores of Y (register path); bit 2: same for the TMA stores
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
@@ -678,23 +678,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     st_shared_v4(box_row + ((j ^ (lane & 7)) << 4), v[0], v[1], v[2], v[3]);
                 };
                 auto issue = [&](int h) {
-                    if (p.y_tma == 2) {
-                        // the warp copies its box to Y: 8 lanes per 128-byte
-                        // box row, 4 rows per instruction (the TMA unit keeps
-                        // to the operand loads)
-                        __syncwarp();
-                        const int ch = lane & 7;
-                        const int col = colh + h * 64 + ch * 8;
-#pragma unroll
-                        for (int it = 0; it < 8; ++it) {
-                            const int rr = it * 4 + (lane >> 3);
-                            const uint4 v = ld_shared_v4(smem_u32(box) + rr * 128 + ((ch ^ (rr & 7)) << 4));
-                            if (row0 + rr < p.M && col < p.N)
-                                *reinterpret_cast<uint4*>(p.y + (int64_t)(row0 + rr) * p.N + col) = v;
-                        }
-                        __syncwarp();
-                        return;
-                    }
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0 && row0 < p.M && colh + h * 64 < p.N) {
@@ -970,7 +953,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     memset(&msfb, 0, sizeof(msfb));
     // the SwiGLU form writes H [M, inter] (inter = N / 2) by TMA stores
     const int64_t n_out = SWIGLU ? a.swiglu_inter : a.N;
-    const int y_mode = SWIGLU ? 1 : env_int("MQ_GEMM_YTMA", 0, 2, 1);
+    const int y_mode = SWIGLU ? 1 : env_int("MQ_GEMM_YTMA", 0, 1, 1);
     const bool y_tma = C::TMA_STORE && y_mode != 0 && make_y_map(&my, a.y, a.M, n_out);
     bool sfb_tma;
     if (SWIGLU) {
