@@ -105,6 +105,16 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmap_w);
         prefetch_tmap(&tmap_x);
+        // This CTA's weight codes and scales start toward L2 before the wait
+        // for the previous grid: a prefetch leaves nothing visible (L2 is the
+        // point of coherence, later writes by that grid still win), and the
+        // weight stream overlaps the previous kernel's tail.
+        const int64_t wt = min(n0 / ROWS, p.w_row_tiles - 1);
+        for (int kt = kt0; kt < kt1; ++kt) {
+            tma_prefetch_2d(&tmap_w, kt * 128, n0);
+            const int nkb = min(NKB, p.kblocks - kt * NKB);
+            bulk_prefetch_l2(p.w_scales + (wt * p.katoms + (int64_t)kt * NKB) * 512, nkb * 512);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&s->tmem_base, TMEM_COLS);
@@ -280,10 +290,13 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stre
     p.status = a.status;
     p.timeout = a.timeout_cycles;
     const int tiles = (int)((a.N + ROWS - 1) / ROWS);
-    // split-K: the smallest power of two (<= 8) that gives about two CTAs per
-    // SM, and never more parts than K stages
+    // split-K: the largest power of two (<= 8) that keeps the grid within one
+    // wave of two CTAs per SM and gives every CTA at least 4 K stages (a
+    // partial second wave, or CTAs of 1-2 stages whose set-up and cluster
+    // reduction outweigh their loads, measured slower on every Qwen3-8B
+    // projection)
     int split = 1;
-    while (split < 8 && (int64_t)tiles * split < 2 * (int64_t)num_sms && split * 2 <= p.k_stages) split *= 2;
+    while (split < 8 && (int64_t)tiles * split * 2 <= 2 * (int64_t)num_sms && p.k_stages >= 4 * split * 2) split *= 2;
     const char* sv = getenv("MQ_DECODE_SPLIT");
     if (sv) {
         const int f = atoi(sv);
