@@ -545,6 +545,35 @@ def _e2e(args, work, device, stream):
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 
+def profile_target(which: str):
+    """One gate/up-shaped NVFP4 GEMM (8192 x 24576 x 4096) inside an NVTX
+    range "gemm", after 3 unmarked launches, for `ncu --nvtx --nvtx-include
+    gemm/`: `ours` is mq_nvfp4_gemm on quantized operands, `library` the
+    library NVFP4 GEMM (cuBLASLt through torch._scaled_mm; context for the
+    profile comparison only, on random codes and unit scales)."""
+    M, N, K = TOKENS, 24576, 4096
+    if which == "library":
+        a = torch.randint(0, 255, (M, K // 2), dtype=torch.uint8, device="cuda").view(torch.float4_e2m1fn_x2)
+        b = torch.randint(0, 255, (N, K // 2), dtype=torch.uint8, device="cuda").view(torch.float4_e2m1fn_x2)
+        sa = torch.full((M * K // 16,), 1.0, device="cuda").to(torch.float8_e4m3fn)
+        sb = torch.full((N * K // 16,), 1.0, device="cuda").to(torch.float8_e4m3fn)
+        f = lambda: torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16)
+    else:
+        from nvfp4_w4a4_quantized_03_b200 import mq
+        x = inputs.activation_bf16(M, K, seed=1, outlier_channels=inputs.outlier_count(K), device="cuda")
+        w = inputs.weight_bf16(N, K, seed=2, device="cuda")
+        qx, qw = mq.quantize(x), mq.quantize(w)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        f = lambda: mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, qw.codes, qw.scales, qw.alpha, M, N, K, y)
+    for _ in range(3):
+        f()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("gemm")
+    f()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -554,7 +583,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sequence", action="store_true",
                     help="skip the 36-layer x 131072-token prefill-sequence, decode and MLP figures")
+    ap.add_argument("--profile-target", choices=["ours", "library"], default=None,
+                    help="run one gate/up GEMM in an NVTX range for ncu and exit (no timing)")
     args = ap.parse_args()
+    if args.profile_target:
+        profile_target(args.profile_target)
+        return
     assert args.warmup >= 3, "at least 3 warm-up steps"
     world, rank, local = _dist()
     try:
