@@ -130,8 +130,6 @@ struct Params {
     long long timeout;
     int fault_skip_first_load;
     int y_tma;               // Y is written by TMA stores (tmap_y is valid)
-    int pf_dist;             // L2 prefetch distance in stages (0: none)
-    int hints;               // bit 1: evict-first stores of Y (register path); bit 2: same for the TMA stores
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
     int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
     int sfb_tma;             // B's two scale slices of a stage arrive as one TMA box (tmap_sfb is valid)
@@ -369,19 +367,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         }
                         pending |= 1u << st;
                         pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
-                    }
-                    if (p.pf_dist > 0) {
-                        // warm L2 with the stage pf_dist ahead (of this tile or a later one)
-                        int kt2 = kt + p.pf_dist, tile2 = tile;
-                        while (kt2 >= p.k_stages) { kt2 -= p.k_stages; tile2 += units; }
-                        if (tile2 < p.tiles) {
-                            int mb2, nb2;
-                            tile_coords(tile2, p, mb2, nb2);
-                            const int arow2 = mb2 * C::TILE_M + (int)rank * BM;
-                            const int brow2 = SWIGLU ? (int)rank * p.inter + nb2 * 128 : nb2 * BN + (int)rank * C::B_ROWS;
-                            tma_prefetch_2d(&tmap_b, kt2 * C::ROW_BYTES, brow2);
-                            if (!QUANT) tma_prefetch_2d(&tmap_a, kt2 * C::ROW_BYTES, arow2);
-                        }
                     }
                     if (++st == p.stages) { st = 0; phase ^= 1; }
                 }
@@ -681,8 +666,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0 && row0 < p.M && colh + h * 64 < p.N) {
-                        if (p.hints & 4) tma_store_2d_hint(&tmap_y, box, colh + h * 64, row0, policy_evict_first());
-                        else tma_store_2d(&tmap_y, box, colh + h * 64, row0);
+                        tma_store_2d(&tmap_y, box, colh + h * 64, row0);
                         bulk_commit_group();
                     }
                 };
@@ -742,25 +726,12 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
                 if (row < p.M) {
                     uint4* d4 = reinterpret_cast<uint4*>(p.y + (int64_t)row * p.N + colh);
-                    if (p.hints & 2) {
-                        // Y is not read again here: let it leave L2 before A and B
-                        const uint64_t pol = policy_evict_first();
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
+                    for (int c = 0; c < 4; ++c)
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                st_global_hint(d4 + c * 4 + j,
-                                               make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
-                                                          packed[c][4 * j + 2], packed[c][4 * j + 3]),
-                                               pol);
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                d4[c * 4 + j] = make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
-                                                           packed[c][4 * j + 2], packed[c][4 * j + 3]);
-                    }
+                        for (int j = 0; j < 4; ++j)
+                            d4[c * 4 + j] = make_uint4(packed[c][4 * j], packed[c][4 * j + 1],
+                                                       packed[c][4 * j + 2], packed[c][4 * j + 3]);
                 }
             } else {
                 // Ragged right edge (or N not a multiple of 8): one 32-column
@@ -993,8 +964,6 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.y_tma = y_tma ? y_mode : 0;
     p.sfb_tma = sfb_tma ? 1 : 0;
     p.sfa_tma = sfa_tma ? 1 : 0;
-    p.pf_dist = env_int("MQ_GEMM_PF", 0, 64, 0);
-    p.hints = env_int("MQ_GEMM_HINTS", 0, 7, 0);
     p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
     p.stages = env_int("MQ_GEMM_STAGES", 2, C::STAGES, C::STAGES);
     p.x = static_cast<const uint16_t*>(a.x);
