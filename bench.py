@@ -281,6 +281,7 @@ def run_ours(args, world, rank, local):
     del work
     torch.cuda.empty_cache()
     sequence = None if args.no_sequence else _prefill_sequence(args, device)
+    sequence_mlp = None if args.no_sequence else _prefill_sequence(args, device, mlp=True)
     decode = None if args.no_sequence else _decode_figure(device)
     mlp = None if args.no_sequence else _mlp_figure(device)
 
@@ -316,6 +317,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.summary(),
         "e2e": e2e,
         "prefill_sequence": sequence,
+        "prefill_sequence_mlp": sequence_mlp,
         "decode_gemm": decode,
         "mlp": mlp,
     }
@@ -392,15 +394,17 @@ def _gemm_pass(args, work, device, stream):
             "ms_per_launch": total_ms / len(bufs)}
 
 
-def _prefill_sequence(args, device):
+def _prefill_sequence(args, device, mlp=False):
     """The 36-layer decoder stack's prefill linears at 131072 tokens (four
     Qwen3-8B-shaped projections per layer, fixed activations, weights
     N(0, 0.02) quantized offline), recorded once as a CUDA graph and replayed;
-    CUDA events around each replay."""
+    CUDA events around each replay.  With `mlp`, each layer's gate/up and
+    down linears are its MLP in one mq_mlp_w4a4 call (SwiGLU and H's
+    quantization between them), the same GEMM flops."""
     from nvfp4_w4a4_quantized_03_b200 import mq
     from nvfp4_w4a4_quantized_03_b200.sequence import PrefillSequence
     layers, tokens = 36, 131072
-    seq = PrefillSequence(layers, tokens, device)
+    seq = PrefillSequence(layers, tokens, device, mlp=mlp)
     seq.capture()
     seq.replay()                      # warm-up
     torch.cuda.synchronize()
@@ -414,9 +418,10 @@ def _prefill_sequence(args, device):
     torch.cuda.synchronize()
     assert seq.status() == mq.MQ_OK
     ms = min(e0.elapsed_time(e1) for e0, e1 in evs)
-    out = {"workload": f"{layers} layers x (qkv, o, gate_up, down) at {tokens} tokens, one CUDA graph",
+    what = "(qkv, o, MLP: gate/up + SwiGLU + down)" if mlp else "(qkv, o, gate_up, down)"
+    out = {"workload": f"{layers} layers x {what} at {tokens} tokens, one CUDA graph",
            "tflops": seq.flops() / (ms / 1e3) / 1e12, "ms": ms, "ms_per_layer": ms / layers,
-           "tflop_per_layer": seq.flops() / layers / 1e12, "graph_kernel_launches": 2 * 4 * layers,
+           "tflop_per_layer": seq.flops() / layers / 1e12, "graph_kernel_launches": seq.launches(),
            "replays_timed": reps, "timing": "best of the timed replays"}
     del seq
     torch.cuda.empty_cache()

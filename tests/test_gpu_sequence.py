@@ -2,7 +2,9 @@
 a CUDA-graph replay gives the eager result bit for bit, the shared workspace
 reports no device error, and a projection of the last layer matches the
 oracle on sampled rows (NVFP4 W4A4 linear, "Mix-Quant：面向智能体LLM的量化预填充
-与精确解码", section 方法步骤详情, step (3))."""
+与精确解码", section 方法步骤详情, step (3)).  With the fused MLP, the last
+layer's MLP output matches the oracle's MLP chain (readings R11-R13 of the
+oracle for the activation between the two linears)."""
 import numpy as np
 import pytest
 import torch
@@ -41,3 +43,31 @@ def test_graph_replay_matches_eager_and_oracle():
     ref = oracle.bf16_rne_array(oracle.gemm_f64(oracle.dequantize(xc, xs, ax), oracle.dequantize(wc, wsc, aw)))
     got = bits(seq.y[i])[rows]
     assert rel_frobenius(bf16_bits_to_f64(got), bf16_bits_to_f64(ref)) <= 1e-3
+
+
+def test_graph_replay_with_fused_mlp():
+    seq = PrefillSequence(layers=2, tokens=640, device=dev(), mlp=True)
+    seq.run()
+    torch.cuda.synchronize()
+    eager = [None if y is None else bits(y) for y in seq.y]
+    seq.capture()
+    for y in seq.y:
+        if y is not None:
+            y.fill_(float("nan"))
+    seq.replay()
+    torch.cuda.synchronize()
+    assert seq.status() == mq.MQ_OK
+    for e, y in zip(eager, seq.y):
+        if y is not None:
+            assert np.array_equal(bits(y), e)
+    assert seq.launches() == 2 * (2 * 2 + 5)
+    # the last layer's MLP (gate/up weight seed index 2, down index 3) against the oracle
+    names = [p.name for p in inputs.QWEN3_8B_PROJECTIONS]
+    igu, idn = names.index("gate_up"), names.index("down")
+    pgu, pdn = inputs.QWEN3_8B_PROJECTIONS[igu], inputs.QWEN3_8B_PROJECTIONS[idn]
+    last = seq.layers - 1
+    wgu = bits(inputs.weight_bf16(pgu.N, pgu.K, seed=1000 + 16 * last + igu, device="cuda"))
+    wdn = bits(inputs.weight_bf16(pdn.N, pdn.K, seed=1000 + 16 * last + idn, device="cuda"))
+    ref = oracle.mlp_w4a4(bits(seq.x[igu]), wgu, wdn)
+    got = bits(seq.y[idn])
+    assert rel_frobenius(bf16_bits_to_f64(got), bf16_bits_to_f64(ref["y_bf16"])) <= 1e-3
