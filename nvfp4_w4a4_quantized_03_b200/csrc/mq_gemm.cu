@@ -162,32 +162,64 @@ struct Smem {
 // (x = k ln2 + r with ln2 split into a 16-bit head and a tail, |r| <= ln2/2)
 // and the Taylor polynomial of e^r to degree 7, each step one IEEE binary32
 // operation; +inf above 88, 0 below -87 (2^k stays a normal number).
-__device__ __forceinline__ float exp_cw(float x) {
-    if (x > 88.0f) return __int_as_float(0x7f800000);
-    if (x < -87.0f) return 0.0f;
-    const float k = rintf(__fmul_rn(x, 0x1.715476p+0f));
-    float r = __fmaf_rn(-k, 0x1.62e4p-1f, x);
-    r = __fmaf_rn(-k, 0x1.7f7d1cp-20f, r);
-    float e = 0x1.a01a02p-13f;
-    e = __fmaf_rn(e, r, 0x1.6c16c2p-10f);
-    e = __fmaf_rn(e, r, 0x1.111112p-7f);
-    e = __fmaf_rn(e, r, 0x1.555556p-5f);
-    e = __fmaf_rn(e, r, 0x1.555556p-3f);
-    e = __fmaf_rn(e, r, 0.5f);
-    e = __fmaf_rn(e, r, 1.0f);
-    e = __fmaf_rn(e, r, 1.0f);
-    return __fmul_rn(e, __int_as_float(((int)k + 127) << 23));
+// Two lanes at once: the binary32 pair instructions (fma.rn.f32x2,
+// mul.rn.f32x2) round each lane exactly as the scalar ones do, so the pair
+// form gives the same bits as the step-by-step definition above.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
-__device__ __forceinline__ float swiglu_f32(float g, float u) {
-    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, exp_cw(-g))), u);
+// e(x0), e(x1): x clamped to [-87, 88] for the arithmetic (2^k normal, k an
+// exact small integer), the out-of-range lanes then set to +inf / 0
+__device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1) {
+    const float c0 = fminf(fmaxf(x0, -87.0f), 88.0f), c1 = fminf(fmaxf(x1, -87.0f), 88.0f);
+    float t0, t1;
+    f2_split(f2_mul(f2(c0, c1), f2(0x1.715476p+0f, 0x1.715476p+0f)), t0, t1);
+    const float k0 = rintf(t0), k1 = rintf(t1);
+    const uint64_t nk = f2(-k0, -k1);
+    uint64_t r = f2_fma(nk, f2(0x1.62e4p-1f, 0x1.62e4p-1f), f2(c0, c1));
+    r = f2_fma(nk, f2(0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f), r);
+    uint64_t e = f2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
+    e = f2_fma(e, r, f2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
+    e = f2_fma(e, r, f2(0x1.111112p-7f, 0x1.111112p-7f));
+    e = f2_fma(e, r, f2(0x1.555556p-5f, 0x1.555556p-5f));
+    e = f2_fma(e, r, f2(0x1.555556p-3f, 0x1.555556p-3f));
+    e = f2_fma(e, r, f2(0.5f, 0.5f));
+    e = f2_fma(e, r, f2(1.0f, 1.0f));
+    e = f2_fma(e, r, f2(1.0f, 1.0f));
+    e = f2_mul(e, f2(__int_as_float(((int)k0 + 127) << 23), __int_as_float(((int)k1 + 127) << 23)));
+    f2_split(e, e0, e1);
+    if (x0 > 88.0f) e0 = __int_as_float(0x7f800000);
+    if (x0 < -87.0f) e0 = 0.0f;
+    if (x1 > 88.0f) e1 = __int_as_float(0x7f800000);
+    if (x1 < -87.0f) e1 = 0.0f;
 }
 
 // two bf16 pairs (g, u packed as bf16x2) -> h packed as bf16x2
 __device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
-    const float h_lo = swiglu_f32(__uint_as_float(g2 << 16), __uint_as_float(u2 << 16));
-    const float h_hi = swiglu_f32(__uint_as_float(g2 & 0xffff0000u), __uint_as_float(u2 & 0xffff0000u));
-    return cvt_bf16x2(h_hi, h_lo);
+    const float g0 = __uint_as_float(g2 << 16), g1 = __uint_as_float(g2 & 0xffff0000u);
+    float e0, e1, d0, d1;
+    exp_cw2(-g0, -g1, e0, e1);
+    f2_split(f2_fma(f2(e0, e1), f2(1.0f, 1.0f), f2(1.0f, 1.0f)), d0, d1);     // 1 + e, one rounding each
+    const uint64_t s = f2(__fdiv_rn(g0, d0), __fdiv_rn(g1, d1));
+    float h0, h1;
+    f2_split(f2_mul(s, f2(__uint_as_float(u2 << 16), __uint_as_float(u2 & 0xffff0000u))), h0, h1);
+    return cvt_bf16x2(h1, h0);
 }
 
 __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
