@@ -34,12 +34,12 @@ METRIC = "W4A4 NVFP4 linear TFLOPS (quant+GEMM) & % of B200 FP4 peak; quant GB/s
 WORKLOAD = "qwen3-8b prefill projections (qkv, o, gate_up, down) at 8192 tokens, NVFP4 W4A4"
 
 
-def _gemm_traffic():
-    """DRAM bytes per k_gemm launch (mean over the four projections) from the
-    committed ncu capture, or None once the kernel's sources have changed
-    since the capture (the counters would describe another kernel)."""
+def _traffic(record: str, key: str):
+    """DRAM bytes from a committed ncu capture (profiles/<record>), or None
+    once the kernels' sources have changed since the capture (the counters
+    would describe other kernels)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "k_gemm_dram_traffic.json")
+    path = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -50,7 +50,18 @@ def _gemm_traffic():
             h.update(f.read())
     if h.hexdigest()[:16] != rec["sources_sha256_16"]:
         return None
-    return rec["mean_per_launch_bytes"]
+    return rec[key]
+
+
+def _gemm_traffic():
+    """DRAM bytes per k_gemm launch, mean over the four projections."""
+    return _traffic("k_gemm_dram_traffic.json", "mean_per_launch_bytes")
+
+
+def _quant_traffic():
+    """DRAM bytes of the stand-alone quantizer per activation (k_amax +
+    k_quantize_tiles), mean over the four activations."""
+    return _traffic("quant_dram_traffic.json", "mean_per_activation_bytes")
 
 
 def _peaks():
@@ -310,7 +321,9 @@ def run_ours(args, world, rank, local):
                             "frac": lin_tflops / fp4_peak,
                             "kernel": "mq_linear_w4a4 = k_quantize_onepass_tiles + k_gemm"},
         "quant_roofline": {"bound": "hbm", "achieved": quant["gbs"], "peak": hbm, "unit": "GB/s",
-                           "frac": quant["gbs"] / hbm, "traffic": None,
+                           "frac": quant["gbs"] / hbm, "traffic": _quant_traffic(),
+                           "traffic_unit": "bytes per activation (k_amax + k_quantize_tiles; mean of the four "
+                                           "activations, algorithmic 4.5625 B/element = 211.8 MB; ncu dram read+write)",
                            "kernel": "k_amax + k_quantize_tiles (mq_tensor_scale + mq_nvfp4_quantize)",
                            "bytes_per_element": 4.5625, "peak_source": f"{peaks_src}: hbm_gbs"},
         "gpu_launches": 8 * args.steps,
