@@ -248,7 +248,8 @@ int mq_read_status(void *ws, void *stream, int32_t *device_status);
 
 /*
  * Failure-detection test hook; the paper has no counterpart.  Runs the
- * mq_nvfp4_gemm kernel with the loads of the first pipeline stage withheld
+ * mq_nvfp4_gemm kernel (the decode form for M <= 64) with the loads of the
+ * first pipeline stage withheld
  * and every bounded wait limited to `timeout_cycles` SM clock cycles
  * (1e5 .. 4e9), so the pipeline stalls on purpose: each waiting role gives
  * up, the kernel writes MQ_ERR_TIMEOUT into the workspace status word, lets

@@ -60,6 +60,7 @@ struct Params {
     int kblocks, k_stages, katoms, w_row_tiles, split;
     int* status;
     long long timeout;
+    int fault_skip_first_load;   // failure-detection test hook: withhold the first stage's copies
 };
 
 struct Smem {
@@ -138,17 +139,38 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             const int64_t wt = min(n0 / ROWS, p.w_row_tiles - 1);
             int st = 0;
             uint32_t phase = 0;
+            uint32_t pending = 0, pending_phase = 0;     // stages with copies in flight, and their parity
+            bool skip = p.fault_skip_first_load != 0;
             for (int kt = kt0; kt < kt1; ++kt) {
                 if (!mbar_wait_bounded(&s->empty[st], phase ^ 1, p.timeout, abort_flag)) { raise(); break; }
-                const int nkb = min(NKB, p.kblocks - kt * NKB);
-                const int64_t ka = (int64_t)kt * NKB;
-                mbar_arrive_expect_tx(&s->ready[st], W_BYTES + p.MP * 128);
-                tma_load_2d(stage_w(st), &tmap_w, &s->ready[st], kt * 128, n0);
-                tma_load_2d(stage_x(st), &tmap_x, &s->ready[st], kt * 128, 0);
-                mbar_arrive_expect_tx(&s->sf_full[st], 2 * nkb * 512);
-                bulk_load(stage_sfw(st), p.w_scales + (wt * p.katoms + ka) * 512, nkb * 512, &s->sf_full[st]);
-                bulk_load(stage_sfx(st), p.x_scales + ka * 512, nkb * 512, &s->sf_full[st]);
+                pending &= ~(1u << st);
+                if (skip) {
+                    skip = false;       // this stage never completes: every wait on it runs out
+                } else {
+                    const int nkb = min(NKB, p.kblocks - kt * NKB);
+                    const int64_t ka = (int64_t)kt * NKB;
+                    mbar_arrive_expect_tx(&s->ready[st], W_BYTES + p.MP * 128);
+                    tma_load_2d(stage_w(st), &tmap_w, &s->ready[st], kt * 128, n0);
+                    tma_load_2d(stage_x(st), &tmap_x, &s->ready[st], kt * 128, 0);
+                    mbar_arrive_expect_tx(&s->sf_full[st], 2 * nkb * 512);
+                    bulk_load(stage_sfw(st), p.w_scales + (wt * p.katoms + ka) * 512, nkb * 512, &s->sf_full[st]);
+                    bulk_load(stage_sfx(st), p.x_scales + ka * 512, nkb * 512, &s->sf_full[st]);
+                    pending |= 1u << st;
+                    pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
+                }
                 if (++st == STAGES) { st = 0; phase ^= 1; }
+            }
+            if (*abort_flag) {
+                // the copies this thread issued land before the CTA releases
+                // its shared memory: a stage's scale copies complete its
+                // sf_full barrier by themselves, its code tiles (issued just
+                // before them) get a short grace period
+                for (int i = 0; i < STAGES; ++i)
+                    if (pending & (1u << i))
+                        mbar_wait_bounded(&s->sf_full[i], (pending_phase >> i) & 1, p.timeout, nullptr);
+                const long long t0 = clock64();
+                while (clock64() - t0 < 200000) {
+                }
             }
         }
     } else if (warp == 1) {
@@ -259,7 +281,7 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 // ---------------------------------------------------------------- host side
 cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     using namespace decode;
-    if (a.x || a.fault_skip_first_load || a.M < 1 || a.M > MP_MAX) return cudaErrorNotSupported;
+    if (a.x || a.M < 1 || a.M > MP_MAX) return cudaErrorNotSupported;
     const int MP = (int)((a.M + 15) / 16 * 16);
     CUtensorMap mw, mx;
     if (!make_fp4_code_map(&mw, a.b_codes, a.N, a.K, ROWS) || !make_fp4_code_map(&mx, a.a_codes, a.M, a.K, MP))
@@ -289,6 +311,7 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stre
     p.w_row_tiles = (int)(padded_rows(a.N) / 128);
     p.status = a.status;
     p.timeout = a.timeout_cycles;
+    p.fault_skip_first_load = a.fault_skip_first_load;
     const int tiles = (int)((a.N + ROWS - 1) / ROWS);
     // split-K: the largest power of two (<= 8) that keeps the grid within one
     // wave of two CTAs per SM and gives every CTA at least 4 K stages (a

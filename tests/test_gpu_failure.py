@@ -55,6 +55,29 @@ def test_stalled_gemm_reports_timeout_and_context_survives(form, monkeypatch):
     assert rel_frobenius(bf16_bits_to_f64(bits(y)), bf16_bits_to_f64(ref["y_bf16"])) <= 1e-3
 
 
+def test_stalled_decode_gemm_reports_timeout_and_context_survives():
+    """The decode form (M <= 64, split-K over a cluster): every CTA withholds
+    its first stage, all bounded waits run out, the copies already issued land
+    before the CTAs end, and the next decode GEMM is correct."""
+    M, N, K = 8, 1024, 4096
+    x = inputs.activation_bf16(M, K, seed=19, outlier_channels=10).to(dev())
+    w = inputs.weight_bf16(N, K, seed=20).to(dev())
+    qx, qw = mq.quantize(x), mq.quantize(w)
+    ws = mq.workspace(mq.mq_workspace_bytes(), dev())
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = _stall_fn()(_p(qx.codes), _p(qx.scales), _p(qx.alpha), _p(qw.codes), _p(qw.scales), _p(qw.alpha),
+                     M, N, K, _p(y), _p(ws), ws.numel(), 2_000_000, stream)
+    assert st == mq.MQ_OK
+    torch.cuda.synchronize()
+    assert mq.mq_read_status(ws) == mq.MQ_ERR_TIMEOUT
+    mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, qw.codes, qw.scales, qw.alpha, M, N, K, y, ws)
+    torch.cuda.synchronize()
+    assert mq.mq_read_status(ws) == mq.MQ_OK
+    ref = oracle.linear_w4a4(bits(x.cpu()), bits(w.cpu()))
+    assert rel_frobenius(bf16_bits_to_f64(bits(y)), bf16_bits_to_f64(ref["y_bf16"])) <= 1e-3
+
+
 def test_stall_hook_validates_its_limit():
     f = _stall_fn()
     dummy = ctypes.c_void_p(1 << 20)
