@@ -17,10 +17,12 @@
 //              this halves B's shared-memory reads and cuts L2 traffic by a
 //              third against PAIR = 1.
 // Warp roles (both forms):
-//   warp 0      producer: per stage, the block-scale tiles (plain bulk copies,
-//               completing on this CTA's sf_full) and then the A/B code tiles
-//               (TMA, 128-byte swizzle; in the pair form both CTAs' copies
-//               complete on CTA 0's `ready` barrier).
+//   warp 0      producer: per stage, the A/B code tiles (TMA, 128-byte
+//               swizzle; in the pair form both CTAs' copies complete on CTA
+//               0's `ready` barrier), then the block-scale slices as TMA boxes
+//               of the scale array viewed as 64-bit words (A's slice, and B's
+//               two slices in one 2-row box), completing on this CTA's
+//               sf_full: four copies per stage.
 //   warp 1      allocates TMEM; in the (even) CTA one lane issues
 //               tcgen05.mma (K = 64 per instruction, 4 per stage) and
 //               tcgen05.commit to release stages and to publish a tile.
@@ -43,6 +45,11 @@
 //   warps 8..15 epilogue: drain the CTA's 128 x 256 fp32 accumulator into
 //               registers (scaled by alpha_a * alpha_b, rounded to bf16),
 //               release it to the MMA thread, then store.
+// SwiGLU form (pair tiles, mq_nvfp4_gemm_swiglu): B is a [2 inter, K]
+// gate/up weight; CTA 0 stages 128 gate rows and CTA 1 the matching 128 up
+// rows, so each accumulator holds the gate and up products of the same 128
+// output columns; the epilogue rounds both to bf16, applies SwiGLU, writes H
+// and raises the running max|h|.
 // Every wait on an mbarrier is bounded; on a timeout the kernel records
 // MQ_ERR_TIMEOUT in the status word, unwinds every role, waits (bounded) for
 // its own copies and MMAs, frees TMEM and returns.
