@@ -166,7 +166,10 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 }
 // this thread's bulk stores are complete
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// generic-proxy shared-memory writes become visible to the async proxy
+// Orders this thread's generic-proxy shared-memory accesses with later
+// async-proxy ones: writes become visible to a TMA store, and reads are
+// performed before a TMA load that refills the same bytes (a release/acquire
+// chain through an mbarrier alone does not order the two proxies).
 __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -180,6 +180,7 @@ k_quantize_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t
                 v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
             quantize_quad(nullptr, rows, K, (uint32_t)row, kg, alpha, codes, scales, v);
         }
+        fence_proxy_async_shared();   // the reads are performed before the slot's next TMA load
         __syncthreads();     // every thread is done with this box
         if (threadIdx.x == 0 && t + (int64_t)QT_STAGES * gridDim.x < ntiles) issue(t + (int64_t)QT_STAGES * gridDim.x, st);
     }
@@ -293,6 +294,7 @@ k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows,
             const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
             if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
         }
+        fence_proxy_async_shared();   // the reads are performed before the slot's next TMA load
         __syncthreads();     // every thread is done with this box
         if (threadIdx.x == 0 && item + QT_STAGES < 2 * n) issue(item + QT_STAGES);
     }
@@ -300,6 +302,206 @@ k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows,
     if (threadIdx.x == 0 && !ok_shared) {
         const long long t0 = clock64();
         while (clock64() - t0 < 200000) {
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// k_quantize_ws: k_quantize_tiles as a producer/consumer pipeline (one lane
+// of warp 8 streams this block's boxes into the ring as slots free up; warps
+// 0..7 quantize one box row per thread and release a slot with one arrival
+// per warp).  Every wait is bounded.
+constexpr int QW_CONSUMERS = QT_THREADS / 32;
+constexpr int QW_THREADS = QT_THREADS + 32;
+
+__global__ void __launch_bounds__(QW_THREADS, 2)
+k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
+              const float* __restrict__ alpha_p, uint4* __restrict__ codes, uint8_t* __restrict__ scales) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[QT_STAGES], empty[QT_STAGES];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t kgroups = K / 64;
+    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
+    const int64_t n = ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;   // boxes of this block
+    const long long timeout = 4000000000LL;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < QT_STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], QW_CONSUMERS);
+        }
+        fence_mbar_init();
+        prefetch_tmap(&xmap);
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    pdl_wait();
+    if (warp == QW_CONSUMERS) {
+        if (lane == 0) {
+            int64_t i = 0;
+            for (; i < n; ++i) {
+                const int st = (int)(i % QT_STAGES);
+                const uint32_t round = (uint32_t)(i / QT_STAGES);
+                if (round > 0 && !mbar_wait_bounded(&empty[st], (round - 1) & 1, timeout, nullptr)) break;
+                const int64_t t = blockIdx.x + i * gridDim.x;
+                mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
+                tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
+                            (int32_t)(t / kgroups) * QT_ROWS);
+            }
+            // every copy this thread issued lands before the block ends
+            for (int64_t j = i > QT_STAGES ? i - QT_STAGES : 0; j < i; ++j)
+                mbar_wait_bounded(&full[j % QT_STAGES], (uint32_t)(j / QT_STAGES) & 1, timeout, nullptr);
+        }
+        return;
+    }
+    const float alpha = __ldg(alpha_p);
+    for (int64_t i = 0; i < n; ++i) {
+        const int st = (int)(i % QT_STAGES);
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[st], (uint32_t)(i / QT_STAGES) & 1, timeout, nullptr)))
+            break;
+        const uint8_t* src = base + st * QT_BOX_BYTES + threadIdx.x * 128;
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
+        fence_proxy_async_shared();   // the reads are performed before the slot's next TMA load
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);       // this warp is done with the slot
+        const int64_t t = blockIdx.x + i * gridDim.x;
+        const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
+        if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// k_quantize_onepass_ws: the same one-pass quantizer as a producer/consumer
+// pipeline.  One lane of warp 8 streams the boxes into the ring as soon as a
+// slot is free (full/empty mbarriers); warps 0..7 take one box row per thread
+// and release a slot with one arrival per warp, so within a phase no warp
+// waits for another.  At the phase boundary the warps' maxima meet through an
+// mbarrier (one arrival per warp), thread 0 joins the grid barrier, and the
+// warps wait for alpha on a second mbarrier.  Every wait is bounded.
+__global__ void __launch_bounds__(QW_THREADS, 2)
+k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
+                      uint32_t* __restrict__ ws, float* __restrict__ alpha_out, uint4* __restrict__ codes,
+                      uint8_t* __restrict__ scales, int* __restrict__ status, long long timeout) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[QT_STAGES], empty[QT_STAGES], p1_done, alpha_ready;
+    __shared__ uint32_t red[QW_CONSUMERS];
+    __shared__ int ok_shared;
+    __shared__ float alpha_shared;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t kgroups = K / 64;
+    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
+    const int64_t n = ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;   // boxes of this block
+    auto box_of = [&](int64_t item) -> int64_t {   // phase 1: boxes in order; phase 2: the same, reversed
+        const int64_t i = item < n ? item : 2 * n - 1 - item;
+        return blockIdx.x + i * gridDim.x;
+    };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < QT_STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], QW_CONSUMERS);
+        }
+        mbar_init(&p1_done, QW_CONSUMERS);
+        mbar_init(&alpha_ready, 1);
+        fence_mbar_init();
+        prefetch_tmap(&xmap);
+        ok_shared = 1;
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    pdl_wait();
+    if (warp == QW_CONSUMERS) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            int64_t item = 0;
+            for (; item < 2 * n; ++item) {
+                const int st = (int)(item % QT_STAGES);
+                const uint32_t round = (uint32_t)(item / QT_STAGES);
+                if (round > 0 && !mbar_wait_bounded(&empty[st], (round - 1) & 1, timeout, nullptr)) break;
+                const int64_t t = box_of(item);
+                mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
+                tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
+                            (int32_t)(t / kgroups) * QT_ROWS);
+            }
+            // every copy this thread issued lands before the block ends
+            for (int64_t j = item > QT_STAGES ? item - QT_STAGES : 0; j < item; ++j)
+                mbar_wait_bounded(&full[j % QT_STAGES], (uint32_t)(j / QT_STAGES) & 1, timeout, nullptr);
+        }
+        return;
+    }
+    // -------------------------------------------------------------------- consumers
+    const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(&ws[WS_GENERATION]);
+    uint32_t m = 0;
+    float alpha = 0.0f;
+    bool ok = true;
+    auto boundary = [&]() {
+        const uint32_t v = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
+        if (lane == 0) {
+            red[warp] = v;
+            mbar_arrive(&p1_done);
+        }
+        if (threadIdx.x == 0) {
+            bool good = mbar_wait_bounded(&p1_done, 0, timeout, nullptr);
+            if (good) {
+                uint32_t w = 0;
+                for (int k = 0; k < QW_CONSUMERS; ++k) w = max(w, red[k]);
+                atomicMax(&ws[WS_AMAX_BITS], w);
+                __threadfence();
+                const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
+                if (ticket == gridDim.x - 1) {
+                    __threadfence();
+                    const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
+                    atomicExch(&ws[WS_TICKET], 0u);
+                    const float amax = __uint_as_float(bits << 16);
+                    *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                    __threadfence();
+                    atomicAdd(&ws[WS_GENERATION], 1u);
+                } else {
+                    const long long t0 = clock64();
+                    while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
+                        if (clock64() - t0 > timeout) {
+                            good = false;
+                            break;
+                        }
+                    }
+                }
+            }
+            if (!good && status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
+            alpha_shared = good ? *reinterpret_cast<volatile float*>(alpha_out) : 0.0f;
+            ok_shared = good ? 1 : 0;
+            mbar_arrive(&alpha_ready);
+        }
+        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&alpha_ready, 0, timeout, nullptr));
+        alpha = alpha_shared;
+        ok = got && ok_shared != 0;
+    };
+    if (n == 0) boundary();
+    for (int64_t item = 0; ok && item < 2 * n; ++item) {
+        if (item == n) {
+            boundary();
+            if (!ok) break;
+        }
+        const int st = (int)(item % QT_STAGES);
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[st], (uint32_t)(item / QT_STAGES) & 1, timeout, nullptr))) {
+            if (lane == 0 && status) atomicExch(status, -7);
+            break;
+        }
+        const uint8_t* src = base + st * QT_BOX_BYTES + threadIdx.x * 128;
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
+        fence_proxy_async_shared();   // the reads are performed before the slot's next TMA load
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);       // this warp is done with the slot
+        if (item < n) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m = absmax_vec(m, v[j]);
+        } else {
+            const int64_t t = box_of(item);
+            const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
+            if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
         }
     }
 }
@@ -417,17 +619,33 @@ cudaError_t launch_quantize_onepass(const void* x, int64_t rows, int64_t K, uint
         }
         // every block resident (grid barrier) and every block owning at least one box
         const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * tiles_per_sm[d]));
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
-        cfg.gridDim = dim3(grid);
-        cfg.blockDim = dim3(QT_THREADS);
         cfg.dynamicSmemBytes = QT_SMEM;
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        const char* wv = getenv("MQ_ONEPASS_WS");
+        if (!(wv && wv[0] == '0')) {
+            // the producer/consumer form (MQ_ONEPASS_WS=0: the block-synchronous ring)
+            static int ws_per_sm[64] = {};
+            if (!ws_per_sm[d]) {
+                cudaError_t e = cudaFuncSetAttribute(k_quantize_onepass_ws, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     QT_SMEM);
+                if (e != cudaSuccess) return e;
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ws_per_sm[d], k_quantize_onepass_ws, QW_THREADS,
+                                                                  QT_SMEM);
+                if (e != cudaSuccess || ws_per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+            }
+            cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * ws_per_sm[d])));
+            cfg.blockDim = dim3(QW_THREADS);
+            return cudaLaunchKernelEx(&cfg, k_quantize_onepass_ws, xmap, rows, prows, K, ws_words, alpha_out,
+                                      reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
+        }
+        cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * tiles_per_sm[d])));
+        cfg.blockDim = dim3(QT_THREADS);
         return cudaLaunchKernelEx(&cfg, k_quantize_onepass_tiles, xmap, rows, prows, K, ws_words, alpha_out,
                                   reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
     }
@@ -505,6 +723,8 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
             cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
             cudaError_t e = cudaFuncSetAttribute(k_quantize_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
             if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(k_quantize_ws, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
+            if (e != cudaSuccess) return e;
             attr_set[d] = true;
         }
         const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
@@ -514,11 +734,18 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
         int nattr = 0;
         set_pdl_attr(attr, &nattr);
         cfg.gridDim = dim3(grid);
-        cfg.blockDim = dim3(QT_THREADS);
         cfg.dynamicSmemBytes = QT_SMEM;
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = nattr;
+        const char* wv = getenv("MQ_QUANT_WS");
+        if (!(wv && wv[0] == '0')) {
+            // the producer/consumer form (MQ_QUANT_WS=0: the block-synchronous ring)
+            cfg.blockDim = dim3(QW_THREADS);
+            return cudaLaunchKernelEx(&cfg, k_quantize_ws, xmap, rows, prows, K, alpha,
+                                      reinterpret_cast<uint4*>(codes), scales);
+        }
+        cfg.blockDim = dim3(QT_THREADS);
         return cudaLaunchKernelEx(&cfg, k_quantize_tiles, xmap, rows, prows, K, alpha, reinterpret_cast<uint4*>(codes),
                                   scales);
     }
