@@ -60,7 +60,7 @@ def _gemm_traffic():
 
 def _quant_traffic():
     """DRAM bytes of the stand-alone quantizer per activation (k_amax +
-    k_quantize_tiles), mean over the four activations."""
+    k_quantize_ws), mean over the four activations."""
     return _traffic("quant_dram_traffic.json", "mean_per_activation_bytes")
 
 
@@ -319,12 +319,12 @@ def run_ours(args, world, rank, local):
                      "peak_source": f"{peaks_src}: 4 x bf16_tflops_sustained (nominal fp4:bf16 = 4)"},
         "linear_roofline": {"bound": "tensor", "achieved": lin_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                             "frac": lin_tflops / fp4_peak,
-                            "kernel": "mq_linear_w4a4 = k_quantize_onepass_tiles + k_gemm"},
+                            "kernel": "mq_linear_w4a4 = k_quantize_onepass_ws + k_gemm"},
         "quant_roofline": {"bound": "hbm", "achieved": quant["gbs"], "peak": hbm, "unit": "GB/s",
                            "frac": quant["gbs"] / hbm, "traffic": _quant_traffic(),
-                           "traffic_unit": "bytes per activation (k_amax + k_quantize_tiles; mean of the four "
+                           "traffic_unit": "bytes per activation (k_amax + k_quantize_ws; mean of the four "
                                            "activations, algorithmic 4.5625 B/element = 211.8 MB; ncu dram read+write)",
-                           "kernel": "k_amax + k_quantize_tiles (mq_tensor_scale + mq_nvfp4_quantize)",
+                           "kernel": "k_amax + k_quantize_ws (mq_tensor_scale + mq_nvfp4_quantize)",
                            "bytes_per_element": 4.5625, "peak_source": f"{peaks_src}: hbm_gbs"},
         "gpu_launches": 8 * args.steps,
         "clocks": clocks.summary(),

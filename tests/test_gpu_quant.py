@@ -109,3 +109,34 @@ def test_rounding_midpoints_sweep():
     for k in range(-4, 5):
         alpha = float(np.float32(2.0 ** -4) * np.float32(1 + k * 2.0 ** -23))
         assert_quant_matches(x, alpha=alpha)
+
+
+@pytest.mark.slow
+def test_repeated_runs_match_the_oracle():
+    """The quantizers stream X through a ring of shared-memory slots that TMA
+    refills while other warps still quantize: repeated runs on an activation
+    that gives each block ~20 boxes (8192 x 12288) must all match the
+    oracle, every L2 state included (a flush before every other run), and the
+    linear's one-pass quantizer must give the same Y every time."""
+    rows, K = 8192, 12288
+    x_cpu = inputs.activation_bf16(rows, K, seed=77, outlier_channels=inputs.outlier_count(K), outlier_scale=50.0)
+    a0, codes0, scales0 = assert_quant_matches(x_cpu)
+    x = x_cpu.to(dev())
+    q = mq.QuantizedTensor(rows, K, dev())
+    q.alpha.fill_(a0)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev())
+    for r in range(12):
+        if r % 2:
+            flush.sum()
+        q.codes.zero_()
+        mq.mq_nvfp4_quantize(x, q.alpha, q.codes, q.scales)
+        torch.cuda.synchronize()
+        assert np.array_equal(q.codes.cpu().numpy().reshape(rows, K // 2), codes0), r
+        assert np.array_equal(q.scales.cpu().numpy(), scales0), r
+    lin = mq.LinearW4A4(inputs.weight_bf16(1024, K, seed=78, device=dev()))
+    y0 = lin(x).clone()
+    for r in range(12):
+        if r % 2:
+            flush.sum()
+        assert torch.equal(lin(x).view(torch.int16), y0.view(torch.int16)), r
+    assert mq.mq_read_status(lin._ws) == mq.MQ_OK
