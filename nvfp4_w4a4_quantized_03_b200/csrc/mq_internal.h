@@ -14,9 +14,10 @@ enum WsWord : int {
     WS_TICKET = 1,      // blocks of the amax pass that have finished
     WS_STATUS = 2,      // device-side status (0 = ok, else an mq_status code)
     WS_ALPHA = 3,       // alpha_x written by the amax pass of mq_linear_w4a4
-    WS_GENERATION = 4,  // grid-barrier generation of the one-pass quantizer (only grows)
     WS_H_AMAX = 5,      // mq_mlp_w4a4: running max of |h| (binary32 bits), zeroed once read
     WS_H_ALPHA = 6,     // mq_mlp_w4a4: alpha_h of the down projection's input
+    WS_GENERATION = 32, // grid-barrier generation of the one-pass quantizer (only grows); a 128-byte
+                        // line of its own, so the blocks polling it do not queue the counters' atomics
 };
 constexpr size_t WS_HEADER_BYTES = 256;
 

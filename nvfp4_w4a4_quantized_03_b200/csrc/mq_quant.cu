@@ -27,6 +27,38 @@ namespace mq {
 
 constexpr int AMAX_THREADS = 512;
 
+// Grid barrier of the one-pass quantizers, taken by one thread per block
+// with its block's max |x| (bf16 bit pattern) `w`: the max joins the
+// workspace's running max, and the last block to arrive (ticket) writes
+// alpha_x, resets the counters and bumps the generation word, which releases
+// the others.  The others poll the generation with a growing sleep (32 ns up
+// to 256 ns), so their loads do not hold up the counters' atomics; the wait
+// gives up after `timeout` cycles (returns false).
+__device__ __forceinline__ bool amax_grid_barrier(uint32_t* ws, uint32_t w, uint32_t gen0, float* alpha_out,
+                                                  long long timeout) {
+    atomicMax(&ws[WS_AMAX_BITS], w);
+    __threadfence();
+    const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
+    if (ticket == gridDim.x - 1) {
+        __threadfence();
+        const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
+        atomicExch(&ws[WS_TICKET], 0u);
+        const float amax = __uint_as_float(bits << 16);
+        *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        __threadfence();
+        atomicAdd(&ws[WS_GENERATION], 1u);
+        return true;
+    }
+    const long long t0 = clock64();
+    unsigned ns = 32;
+    while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
+        if (clock64() - t0 > timeout) return false;
+        __nanosleep(ns);
+        if (ns < 256) ns *= 2;
+    }
+    return true;
+}
+
 // One pass over x (16-byte vectors); every block folds its max into ws with
 // one atomic, and the last block to finish turns it into alpha (or, with
 // raw_amax, writes max |x| itself) and resets the two counters to zero.
@@ -244,26 +276,9 @@ k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows,
         if (threadIdx.x == 0) {
             uint32_t w = 0;
             for (int k = 0; k < QT_THREADS / 32; ++k) w = max(w, red[k]);
-            atomicMax(&ws[WS_AMAX_BITS], w);
-            __threadfence();
-            const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
-            if (ticket == gridDim.x - 1) {
-                __threadfence();
-                const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
-                atomicExch(&ws[WS_TICKET], 0u);
-                const float amax = __uint_as_float(bits << 16);
-                *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-                __threadfence();
-                atomicAdd(&ws[WS_GENERATION], 1u);
-            } else {
-                const long long t0 = clock64();
-                while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
-                    if (clock64() - t0 > timeout) {
-                        ok_shared = 0;
-                        if (status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
-                        break;
-                    }
-                }
+            if (!amax_grid_barrier(ws, w, gen0, alpha_out, timeout)) {
+                ok_shared = 0;
+                if (status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
             }
             alpha_shared = *reinterpret_cast<volatile float*>(alpha_out);
         }
@@ -447,26 +462,7 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
             if (good) {
                 uint32_t w = 0;
                 for (int k = 0; k < QW_CONSUMERS; ++k) w = max(w, red[k]);
-                atomicMax(&ws[WS_AMAX_BITS], w);
-                __threadfence();
-                const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
-                if (ticket == gridDim.x - 1) {
-                    __threadfence();
-                    const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
-                    atomicExch(&ws[WS_TICKET], 0u);
-                    const float amax = __uint_as_float(bits << 16);
-                    *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-                    __threadfence();
-                    atomicAdd(&ws[WS_GENERATION], 1u);
-                } else {
-                    const long long t0 = clock64();
-                    while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
-                        if (clock64() - t0 > timeout) {
-                            good = false;
-                            break;
-                        }
-                    }
-                }
+                good = amax_grid_barrier(ws, w, gen0, alpha_out, timeout);
             }
             if (!good && status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
             alpha_shared = good ? *reinterpret_cast<volatile float*>(alpha_out) : 0.0f;
@@ -544,28 +540,8 @@ k_quantize_onepass(const uint4* __restrict__ x, int64_t rows, int64_t prows, int
     if (threadIdx.x == 0) {
         uint32_t w = 0;
         for (int k = 0; k < ONEPASS_THREADS / 32; ++k) w = max(w, red[k]);
-        atomicMax(&ws[WS_AMAX_BITS], w);
-        __threadfence();
-        const uint32_t ticket = atomicAdd(&ws[WS_TICKET], 1u);
-        bool ok = true;
-        if (ticket == gridDim.x - 1) {
-            __threadfence();
-            const uint32_t bits = atomicExch(&ws[WS_AMAX_BITS], 0u);
-            atomicExch(&ws[WS_TICKET], 0u);
-            const float amax = __uint_as_float(bits << 16);
-            *alpha_out = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-            __threadfence();
-            atomicAdd(&ws[WS_GENERATION], 1u);
-        } else {
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(reinterpret_cast<const int*>(&ws[WS_GENERATION])) == (int)gen0) {
-                if (clock64() - t0 > timeout) {
-                    ok = false;
-                    if (status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
-                    break;
-                }
-            }
-        }
+        const bool ok = amax_grid_barrier(ws, w, gen0, alpha_out, timeout);
+        if (!ok && status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
         ok_shared = ok;
     }
     __syncthreads();
