@@ -33,6 +33,13 @@
 namespace mq {
 namespace decode {
 
+// A cluster barrier that orders no memory accesses: every CTA has reached
+// it, nothing more, so a CTA does not wait here for its own global stores to
+// drain.
+__device__ __forceinline__ void cluster_sync_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
 constexpr int ROWS = 128;            // B rows per CTA (the MMA's M)
 constexpr int MP_MAX = 64;           // tokens per launch (the MMA's N, padded to 16)
 constexpr int STAGES = 3;
@@ -269,7 +276,10 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
     }
     __syncthreads();
-    cluster_sync();     // every CTA keeps its shared memory until all have read it
+    // every CTA keeps its shared memory until all have read it; the reads
+    // have completed (their values went into Y), so the barrier needs no
+    // memory ordering and does not wait for the Y stores
+    cluster_sync_relaxed();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
