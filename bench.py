@@ -295,6 +295,7 @@ def run_ours(args, world, rank, local):
     sequence_mlp = None if args.no_sequence else _prefill_sequence(args, device, mlp=True)
     decode = None if args.no_sequence else _decode_figure(device)
     mlp = None if args.no_sequence else _mlp_figure(device)
+    scale_stats = None if args.no_sequence else _scale_stats(device)
 
     peaks, peaks_src = _peaks()
     fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]        # nominal fp4 : bf16 = 9 : 2.25
@@ -333,6 +334,7 @@ def run_ours(args, world, rank, local):
         "prefill_sequence_mlp": sequence_mlp,
         "decode_gemm": decode,
         "mlp": mlp,
+        "block_scale_stats": scale_stats,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
@@ -488,6 +490,33 @@ def _decode_figure(device):
                         "tflops": 2.0 * M * sum(p.N * p.K for p in projs) / us / 1e6}
         del g
     assert mq.mq_read_status(ws) == mq.MQ_OK
+    return out
+
+
+def _scale_stats(device):
+    """Share of the E4M3 block scales that are zero (the block quantizes to
+    all-zero codes) or subnormal (below 2^-6), on the heavy-tailed long-context
+    activation (32768 x 4096: Student-t(4) times a LogNormal(0, 1) scale per
+    channel) and on the 8192-token activation of the timed step; counted on
+    the quantizer's output scale buffer, outside any timed region."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    out = {}
+    cases = (("student_t_32768x4096", lambda: inputs.student_t_activation_bf16(32768, 4096, seed=300 + 4096,
+                                                                             device=device)),
+             ("gaussian_outliers_8192x4096",
+              lambda: inputs.activation_bf16(TOKENS, 4096, seed=1, outlier_channels=inputs.outlier_count(4096),
+                                             outlier_scale=50.0)))
+    for name, make in cases:
+        x = make().to(device)
+        q = mq.quantize(x)
+        torch.cuda.synchronize()
+        sc = q.scales            # no padding at these shapes: every byte is a block scale
+        n = sc.numel()
+        zero = int((sc == 0).sum().item())
+        sub = int(((sc & 0x78) == 0).sum().item()) - zero
+        out[name] = {"blocks": n, "zero_frac": zero / n, "subnormal_frac": sub / n}
+        del x, q, sc
+    torch.cuda.empty_cache()
     return out
 
 

@@ -70,9 +70,19 @@ def weight_bf16(N: int, K: int, seed: int, std: float = 0.02, device: str = "cpu
     return (torch.randn(N, K, generator=g, dtype=torch.float32, device=device) * std).to(torch.bfloat16)
 
 
-def student_t_activation_bf16(M: int, K: int, seed: int, nu: float = 4.0) -> torch.Tensor:
+def student_t_activation_bf16(M: int, K: int, seed: int, nu: float = 4.0, device: str = "cpu") -> torch.Tensor:
     """Heavy-tailed activations: X[m, k] = s_k * t[m, k], t ~ Student-t(nu),
-    s_k ~ LogNormal(0, 1) per channel (input channel k)."""
+    s_k ~ LogNormal(0, 1) per channel (input channel k).  On the CPU the
+    draws come from numpy's default_rng(seed); on a GPU from a torch generator
+    of that device seeded with `seed` (same distribution, t = z / sqrt(g / nu)
+    with z ~ N(0, 1) and g ~ chi-square(nu) = 2 Gamma(nu / 2), another stream
+    of numbers), for sizes the host would take long to draw."""
+    if str(device) != "cpu":
+        g = torch.Generator(device=device).manual_seed(seed)
+        s = torch.exp(torch.randn(K, generator=g, device=device))
+        z = torch.randn(M, K, generator=g, device=device)
+        chi2 = 2.0 * torch._standard_gamma(torch.full((M, K), nu / 2.0, device=device), generator=g)
+        return (z * torch.rsqrt(chi2 / nu) * s[None, :]).to(torch.bfloat16)
     rng = np.random.default_rng(seed)
     s = rng.lognormal(0.0, 1.0, size=K).astype(np.float32)
     t = rng.standard_t(nu, size=(M, K)).astype(np.float32)
