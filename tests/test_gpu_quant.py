@@ -140,3 +140,24 @@ def test_repeated_runs_match_the_oracle():
             flush.sum()
         assert torch.equal(lin(x).view(torch.int16), y0.view(torch.int16)), r
     assert mq.mq_read_status(lin._ws) == mq.MQ_OK
+
+
+def test_codes_buffer_16_byte_aligned():
+    """A codes buffer that is 16- but not 32-byte aligned (the ABI asks for
+    16) takes the two 128-bit stores per quad instead of one 256-bit store:
+    the same bytes."""
+    rows, K = 640, 1024
+    x_cpu = inputs.activation_bf16(rows, K, seed=91, outlier_channels=10, outlier_scale=50.0)
+    a0, codes0, scales0 = assert_quant_matches(x_cpu)
+    x = x_cpu.to(dev())
+    q = mq.QuantizedTensor(rows, K, dev())
+    q.alpha.fill_(a0)
+    n = mq.mq_nvfp4_codes_bytes(rows, K)
+    buf = torch.zeros(n + 64, dtype=torch.uint8, device=dev())
+    off = 16 if buf.data_ptr() % 32 == 0 else 32      # 16 mod 32 either way
+    codes = buf[off:off + n]
+    assert codes.data_ptr() % 32 == 16
+    mq.mq_nvfp4_quantize(x, q.alpha, codes, q.scales)
+    torch.cuda.synchronize()
+    assert np.array_equal(codes.cpu().numpy().reshape(rows, K // 2), codes0)
+    assert np.array_equal(q.scales.cpu().numpy(), scales0)
