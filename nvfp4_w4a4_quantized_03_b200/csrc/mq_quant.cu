@@ -334,7 +334,11 @@ k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows,
 // k_quantize_ws: k_quantize_tiles as a producer/consumer pipeline (one lane
 // of warp 8 streams this block's boxes into the ring as slots free up; warps
 // 0..7 quantize one box row per thread and release a slot with one arrival
-// per warp).  Every wait is bounded.
+// per warp).  Before a warp releases a slot, each of its threads executes a
+// generic-to-async proxy fence: the mbarrier's release/acquire alone does not
+// order the threads' shared-memory reads before the next TMA write into the
+// slot, and without the fence rows were seen quantized from the next box.
+// Every wait is bounded.
 constexpr int QW_CONSUMERS = QT_THREADS / 32;
 constexpr int QW_THREADS = QT_THREADS + 32;
 
