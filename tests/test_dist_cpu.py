@@ -77,3 +77,48 @@ def test_two_gloo_ranks_share_the_global_amax():
         assert p.exitcode == 0
     got = sorted(q.get(timeout=5) for _ in range(world))
     assert got[0][1] and got[1][1] and got[0][2] == got[1][2]
+
+
+def _column_shard_worker(rank, world, port, q):
+    """Column sharding on the host: each rank holds a block of the weight's
+    rows (a block of Y's columns); the MAX all-reduce of the shards' max|w|
+    gives the whole weight's alpha, under which the oracle's quantization of
+    the rank's rows equals those rows of the whole weight's quantization."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import numpy as np
+    import oracle
+    from nvfp4_w4a4_quantized_03_b200 import inputs
+    from nvfp4_w4a4_quantized_03_b200.sharded import reduce_amax
+    w = inputs.weight_bf16(160, 128, seed=9)
+    w[3, 7] = 0.75             # the largest |w| sits in rank 0's rows only
+    wb = w.contiguous().view(torch.int16).numpy().view(np.uint16)
+    lo, hi = rank * 80, (rank + 1) * 80
+    shard = wb[lo:hi]
+    amax = torch.tensor([float(((np.max(shard.astype(np.uint32) & 0x7FFF)) << 16).astype(np.uint32).view(np.float32))],
+                        dtype=torch.float32)
+    local = float(amax.item())
+    reduce_amax(amax)
+    alpha = float(np.float32(amax.item()) / np.float32(2688.0))
+    whole_alpha = oracle.tensor_scale(wb)
+    codes, scales = oracle.quantize(np.ascontiguousarray(shard), alpha)
+    wc, wsc = oracle.quantize(wb, whole_alpha)
+    q.put((rank, alpha == whole_alpha, bool(np.array_equal(codes, wc[lo:hi]) and np.array_equal(scales, wsc[lo:hi])),
+           local == float(amax.item())))
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_column_shards_match_the_whole_weight():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_column_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    assert all(g[1] and g[2] for g in got), got
+    # rank 1's own max was below the whole weight's: the all-reduce changed it
+    assert got[0][3] and not got[1][3], got
