@@ -22,7 +22,7 @@ import torch
 
 import oracle
 from nvfp4_w4a4_quantized_03_b200 import inputs, mq
-from tests.gpu_helpers import bf16_bits_to_f64, bits, dev, rel_frobenius
+from tests.gpu_helpers import bits, check_gemm_elementwise, dev, linear_ws_codes_rows, linear_ws_scales
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 TOL = 1e-3
@@ -65,11 +65,16 @@ def _check_linear(x_dev: torch.Tensor, w_dev: torch.Tensor, rows: np.ndarray):
     assert float(qx.alpha.item()) == ax
     del qx
     xc, xs = oracle.quantize(np.ascontiguousarray(xb[rows]), ax)
+    # the linear's own quantized activation on those rows, bit for bit
+    ws_codes = linear_ws_codes_rows(lin._ws, M, K, rows)
+    bad = np.argwhere(ws_codes != xc)
+    assert len(bad) == 0, f"{len(bad)} code bytes differ, first {bad[:4].tolist()}"
+    ws_scales = oracle.scales_from_stored(linear_ws_scales(lin._ws, M, K), M, K)[rows]
+    bad = np.argwhere(ws_scales != xs)
+    assert len(bad) == 0, f"{len(bad)} scales differ, first {bad[:4].tolist()}"
     wc, wsc = oracle.quantize(wb, aw)
-    y64 = oracle.gemm_f64(oracle.dequantize(xc, xs, ax), oracle.dequantize(wc, wsc, aw))
-    ref = oracle.bf16_rne_array(y64)
     got = bits(y[torch.from_numpy(rows).to(y.device)])
-    err = rel_frobenius(bf16_bits_to_f64(got), bf16_bits_to_f64(ref))
+    _, err = check_gemm_elementwise(got, oracle.dequantize(xc, xs, ax), oracle.dequantize(wc, wsc, aw), K)
     assert err <= TOL, err
     return err
 

@@ -6,7 +6,8 @@ Y = bf16(xhat . what^T), xhat = alpha sigma q (NVFP4 W4A4, "Mix-Quant：面向
 智能体LLM的量化预填充与精确解码", section 方法步骤详情, step (3); decoding
 quantized as well is the pages' P16D4 variant).  Tolerance: relative
 Frobenius error <= 1e-3 against the oracle's bf16 result on the same
-quantized operands.
+quantized operands, and the per-element bound of
+gpu_helpers.check_elementwise on every output.
 """
 import numpy as np
 import pytest
@@ -14,17 +15,21 @@ import torch
 
 import oracle
 from nvfp4_w4a4_quantized_03_b200 import inputs, mq
-from tests.gpu_helpers import bf16_bits_to_f64, bits, dev, gpu_quantize, rel_frobenius
+from tests.gpu_helpers import bf16_bits_to_f64, bits, check_gemm_elementwise, dev, gpu_quantize, rel_frobenius
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-3
 
 
-def _oracle_y(xb, wb):
+def _check_against_oracle(got, xb, wb):
+    """Per-element bound and relative Frobenius error of a GEMM output against
+    the oracle on the oracle's quantization of (x, w)."""
     ax, aw = oracle.tensor_scale(xb), oracle.tensor_scale(wb)
     xc, xs = oracle.quantize(xb, ax)
     wc, wsc = oracle.quantize(wb, aw)
-    return oracle.bf16_rne_array(oracle.gemm_f64(oracle.dequantize(xc, xs, ax), oracle.dequantize(wc, wsc, aw)))
+    _, err = check_gemm_elementwise(got, oracle.dequantize(xc, xs, ax), oracle.dequantize(wc, wsc, aw),
+                                    xb.shape[1])
+    assert err <= TOL, err
 
 
 def _gemm(M, N, K, x, w):
@@ -48,8 +53,7 @@ def test_decode_gemm_against_oracle(M, N, K, split, monkeypatch):
                                outlier_scale=50.0)
     w = inputs.weight_bf16(N, K, seed=N + 3)
     got = _gemm(M, N, K, x, w)
-    ref = _oracle_y(bits(x), bits(w))
-    assert rel_frobenius(bf16_bits_to_f64(got), bf16_bits_to_f64(ref)) <= TOL
+    _check_against_oracle(got, bits(x), bits(w))
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 12288, 4096), (64, 4096, 12288)])
@@ -62,6 +66,8 @@ def test_decode_matches_prefill_kernel(M, N, K, monkeypatch):
     monkeypatch.setenv("MQ_GEMM_DECODE", "0")
     b = _gemm(M, N, K, x, w)
     assert rel_frobenius(bf16_bits_to_f64(a), bf16_bits_to_f64(b)) <= TOL
+    _check_against_oracle(a, bits(x), bits(w))
+    _check_against_oracle(b, bits(x), bits(w))
 
 
 @pytest.mark.parametrize("M", [1, 8, 64])
@@ -74,5 +80,4 @@ def test_decode_linear(M):
     y = lin(x.to(dev()))
     torch.cuda.synchronize()
     assert mq.mq_read_status(lin._ws) == mq.MQ_OK
-    ref = _oracle_y(bits(x), bits(w))
-    assert rel_frobenius(bf16_bits_to_f64(bits(y)), bf16_bits_to_f64(ref)) <= TOL
+    _check_against_oracle(bits(y), bits(x), bits(w))

@@ -12,7 +12,11 @@ own tensor scale).
     and H, max|h| and H's NVFP4 form must match it bit for bit;
   * tolerance on realistic inputs: H and y within relative Frobenius error
     1e-3 of the oracle's chain (G and U differ from the exact rounding only
-    where the binary32 accumulation crosses a bf16 midpoint);
+    where the binary32 accumulation crosses a bf16 midpoint); per element, H
+    within the bound that G's and U's GEMM bounds imply through the SwiGLU
+    (gpu_helpers.swiglu_bound), and y within the GEMM bound against the
+    oracle's down product of the H the kernel wrote (quantized by the oracle
+    with the kernel's alpha_h);
   * the chain equals the composition of the public calls bit for bit;
   * the Qwen3-8B-shaped MLP at 8192 tokens on sampled rows.
 """
@@ -22,7 +26,8 @@ import torch
 
 import oracle
 from nvfp4_w4a4_quantized_03_b200 import inputs, mq
-from tests.gpu_helpers import bf16_bits_to_f64, bits, dev, rel_frobenius
+from tests.gpu_helpers import (bf16_bits_to_f64, bits, check_elementwise, check_gemm_elementwise, dev,
+                               gemm_bound_terms, rel_frobenius, swiglu_bound)
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-3
@@ -99,6 +104,19 @@ def test_swiglu_gemm_extreme_gate_values():
     assert amax == float(np.max(np.abs(bf16_bits_to_f64(ref))))
 
 
+def _check_h_elementwise(h_bits, g_ref, u_ref, xb, wgub, K, inter, rows=None):
+    """H per element against the oracle's: the gate and up GEMM bounds carried
+    through the SwiGLU (gpu_helpers.swiglu_bound)."""
+    ax, agu = oracle.tensor_scale(xb), oracle.tensor_scale(wgub)
+    xr = xb if rows is None else np.ascontiguousarray(xb[rows])
+    xc, xs = oracle.quantize(xr, ax)
+    gc, gs = oracle.quantize(wgub, agu)
+    _, _, acc = gemm_bound_terms(oracle.dequantize(xc, xs, ax), oracle.dequantize(gc, gs, agu), K)
+    bound = swiglu_bound(g_ref, u_ref, acc[:, :inter], acc[:, inter:])
+    h_ref = oracle.swiglu_bf16(g_ref, u_ref)
+    check_elementwise(h_bits, h_ref, bound, "h")
+
+
 def _mlp_case(M, K, inter, N, seed):
     x = inputs.activation_bf16(M, K, seed=seed, outlier_channels=inputs.outlier_count(K), outlier_scale=50.0,
                                device="cuda")
@@ -120,9 +138,16 @@ def test_mlp_chain_against_oracle(M, K, inter, N):
     assert float(mlp.wgu.alpha.item()) == oracle.tensor_scale(bits(wgu))
     h = bits(mlp.h_view(M))
     assert rel_frobenius(bf16_bits_to_f64(h), bf16_bits_to_f64(ref["h"])) <= TOL
+    _check_h_elementwise(h, ref["g"], ref["u"], bits(x), bits(wgu), K, inter)
     ah = float(mlp._ws[4 * 6:4 * 7].view(torch.float32).item())      # alpha_h word of the workspace header
     assert abs(ah - ref["alpha_h"]) <= ref["alpha_h"] * 2.0 ** -7      # one bf16 step of max|h| at most
     assert rel_frobenius(bf16_bits_to_f64(bits(y)), bf16_bits_to_f64(ref["y_bf16"])) <= TOL
+    # y per element: the down GEMM on the kernel's own H (alpha_h = max|h| / 2688 of that H)
+    assert ah == oracle.tensor_scale(h)
+    hc, hs = oracle.quantize(h, ah)
+    ad = oracle.tensor_scale(bits(wd))
+    dc, ds = oracle.quantize(bits(wd), ad)
+    check_gemm_elementwise(bits(y), oracle.dequantize(hc, hs, ah), oracle.dequantize(dc, ds, ad), inter)
     # the running max was handed on and cleared
     assert int(mlp._ws[4 * 5:4 * 6].view(torch.int32).item()) == 0
 
@@ -172,16 +197,22 @@ def test_qwen3_8b_mlp_8192_tokens_sampled_rows():
     rows = np.unique(np.concatenate([np.random.default_rng(5).choice(M, 32, replace=False), [0, M - 1]]))
     hmax_ref = 0.0
     h_ref_rows = np.empty((len(rows), inter), np.uint16)
+    g_rows = np.empty((len(rows), inter), np.uint16)
+    u_rows = np.empty((len(rows), inter), np.uint16)
     for r0 in range(0, M, 1024):
         y64 = oracle.gemm_f64(oracle.dequantize(xc[r0:r0 + 1024], xs[r0:r0 + 1024], ax), wgu_hat)
-        hc_ = oracle.swiglu_bf16(oracle.bf16_rne_array(y64[:, :inter]), oracle.bf16_rne_array(y64[:, inter:]))
+        g_, u_ = oracle.bf16_rne_array(y64[:, :inter]), oracle.bf16_rne_array(y64[:, inter:])
+        hc_ = oracle.swiglu_bf16(g_, u_)
         hmax_ref = max(hmax_ref, float(np.max(np.abs(bf16_bits_to_f64(hc_)))))
         sel = (rows >= r0) & (rows < r0 + 1024)
         h_ref_rows[sel] = hc_[rows[sel] - r0]
+        g_rows[sel] = g_[rows[sel] - r0]
+        u_rows[sel] = u_[rows[sel] - r0]
     ah_ref = float(np.float32(np.float32(hmax_ref) / np.float32(2688.0)))
     h_all = mlp.h_view(M)
     h_rows = bits(h_all[torch.from_numpy(rows).to(dev())])
     assert rel_frobenius(bf16_bits_to_f64(h_rows), bf16_bits_to_f64(h_ref_rows)) <= TOL
+    _check_h_elementwise(h_rows, g_rows, u_rows, xb, bits(wgu), K, inter, rows)
     ah = float(mlp._ws[24:28].view(torch.float32).item())
     assert abs(ah - ah_ref) <= ah_ref * 2.0 ** -7
     assert ah == float(np.float32(np.float32(float(h_all.abs().max().float().item())) / np.float32(2688.0)))
@@ -191,3 +222,6 @@ def test_qwen3_8b_mlp_8192_tokens_sampled_rows():
     y_ref = oracle.bf16_rne_array(oracle.gemm_f64(oracle.dequantize(hc, hs, ah_ref), oracle.dequantize(dc, ds, ad)))
     y_rows = bits(y[torch.from_numpy(rows).to(dev())])
     assert rel_frobenius(bf16_bits_to_f64(y_rows), bf16_bits_to_f64(y_ref)) <= TOL
+    # y per element: the down GEMM on the kernel's own H rows, quantized with the kernel's alpha_h
+    hk_c, hk_s = oracle.quantize(h_rows, ah)
+    check_gemm_elementwise(y_rows, oracle.dequantize(hk_c, hk_s, ah), oracle.dequantize(dc, ds, ad), inter)
