@@ -57,17 +57,25 @@ class ShardedLinearW4A4:
         self._gemm_ws = mq.workspace(mq.mq_workspace_bytes(), dev)
 
     def __call__(self, x_shard: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Every step runs on `stream` (default: the current stream): the
+        kernels, the all-reduce (torch.distributed orders a collective after
+        the work of the stream that is current when it is called, and the
+        work after it behind it), and the allocations of the call's buffers.
+        The caller orders x_shard's producer (and any given `out`) before
+        `stream`, as for any stream-ordered call."""
         M, K = x_shard.shape
         assert K == self.K
-        mq.mq_tensor_amax(x_shard, self._amax, self._ws, stream)
-        reduce_amax(self._amax, self.group)
-        qx = mq.QuantizedTensor(M, K, x_shard.device)
-        mq.mq_alpha_from_amax(self._amax, qx.alpha, stream)
-        mq.mq_nvfp4_quantize(x_shard, qx.alpha, qx.codes, qx.scales, stream)
-        if out is None:
-            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x_shard.device)
-        mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, self.w.codes, self.w.scales, self.w.alpha, M, self.N, K,
-                         out, self._gemm_ws, stream)
+        s = torch.cuda.current_stream(x_shard.device) if stream is None else stream
+        with torch.cuda.stream(s):
+            mq.mq_tensor_amax(x_shard, self._amax, self._ws)
+            reduce_amax(self._amax, self.group)
+            qx = mq.QuantizedTensor(M, K, x_shard.device)
+            mq.mq_alpha_from_amax(self._amax, qx.alpha)
+            mq.mq_nvfp4_quantize(x_shard, qx.alpha, qx.codes, qx.scales)
+            if out is None:
+                out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x_shard.device)
+            mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, self.w.codes, self.w.scales, self.w.alpha, M, self.N,
+                             K, out, self._gemm_ws)
         return out
 
 
@@ -101,10 +109,12 @@ class ColumnShardedLinearW4A4:
     def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         M, K = x.shape
         assert K == self.K
-        need = mq.mq_linear_w4a4_workspace_bytes(M, K)
-        if self._ws is None or self._ws.numel() < need:
-            self._ws = mq.workspace(need, x.device)
-        if out is None:
-            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
-        mq.mq_linear_w4a4(x, self.w.codes, self.w.scales, self.w.alpha, self.N, out, self._ws, stream)
+        s = torch.cuda.current_stream(x.device) if stream is None else stream
+        with torch.cuda.stream(s):
+            need = mq.mq_linear_w4a4_workspace_bytes(M, K)
+            if self._ws is None or self._ws.numel() < need:
+                self._ws = mq.workspace(need, x.device)
+            if out is None:
+                out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+            mq.mq_linear_w4a4(x, self.w.codes, self.w.scales, self.w.alpha, self.N, out, self._ws)
         return out
