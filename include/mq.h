@@ -228,11 +228,17 @@ int mq_mlp_w4a4(const void *x, int64_t M, int64_t K,
  *   - Shapes whose mq_linear_w4a4_workspace_bytes(M, K) exceeds
  *     MQ_NOALLOC_SCRATCH_BYTES are refused with MQ_ERR_WORKSPACE (e.g.
  *     M = 8192 with K up to 12288 fits; M = 131072, K = 4096 does not).
- *   - The first call on a device looks up the scratch's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - Every call looks up the scratch's device address in the current
+ *     device's current context (cudaGetSymbolAddress), so the address stays
+ *     right after a cudaDeviceReset; the reset itself discards the scratch's
+ *     contents, which no call relies on.  The first call on a device loads
+ *     the library's device code and sets the scratch up: make that first call
+ *     before any stream capture.
  *   - Every call shares the one scratch: calls whose GPU work overlaps (other
  *     streams, other host threads) race and corrupt each other's results;
- *     serialize them.  Each call clears the scratch header before use.
+ *     serialize them.  Each call clears the scratch header before use (one
+ *     cudaMemsetAsync node ahead of the quantizer, which also keeps the next
+ *     call's quantizer from overlapping the previous call's GEMM tail).
  *   - Device-side timeouts land in the scratch's status word, which the caller
  *     cannot read; use mq_linear_w4a4 with a workspace to observe them.
  */

@@ -59,6 +59,11 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA; 
 }  // namespace
 
 namespace mq {
+int check_linear_shape(int64_t M, int64_t N, int64_t K) {
+    const int st = check_rows_k(M, K);
+    return st != MQ_OK ? st : check_rows_k(N, K);
+}
+
 bool pdl_enabled() {
     static int v = -1;
     if (v < 0) {

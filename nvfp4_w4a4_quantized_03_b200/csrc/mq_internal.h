@@ -34,6 +34,10 @@ bool make_bf16_tile_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K
 // box_rows x 128-byte boxes (256 K-elements) in the 128-byte swizzle.
 bool make_fp4_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows);
 
+// The shape checks of mq_linear_w4a4 (rows M and N against K): MQ_OK or
+// MQ_ERR_SHAPE.
+int check_linear_shape(int64_t M, int64_t N, int64_t K);
+
 // Programmatic dependent launch: each kernel lets the next grid on the
 // stream launch early and waits (griddepcontrol.wait) before its first access
 // to global memory.  Launches carry the attribute unless MQ_PDL=0.

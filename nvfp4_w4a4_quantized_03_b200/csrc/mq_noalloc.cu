@@ -11,11 +11,15 @@
 // holds until the process exits.
 //
 // Host code cannot use the array's name as a device address (on the host it
-// names a stand-in object), so the first call on each device, with that
-// device current, looks up the real address with cudaGetSymbolAddress and
-// caches it.  Every call then clears the scratch header and runs the normal
-// mq_linear_w4a4 path with the scratch as its workspace.
-#include <mutex>
+// names a stand-in object), so every call, with the caller's device current,
+// looks up the real address with cudaGetSymbolAddress.  The lookup is cheap
+// once the module is loaded, and doing it per call rather than caching it
+// keeps the address right for the context that is current now: after a
+// cudaDeviceReset the array lives at a new address in a new context.  The
+// first call on a device loads the module and sets the array up, so it
+// should come before any stream capture.  Every call then clears the scratch
+// header and runs the normal mq_linear_w4a4 path with the scratch as its
+// workspace.
 
 #include "../../include/mq.h"
 #include "mq_internal.h"
@@ -24,28 +28,17 @@ namespace {
 
 __device__ __align__(256) uint8_t g_noalloc_scratch[MQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
-int g_scratch_arch_ok[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Device address of the scratch on the current device (set up once per device).
+// Device address of the scratch in the current device's current context.
 int scratch_for_current_device(void** addr) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MQ_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        int major = 0, minor = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-            return MQ_ERR_CUDA;
-        g_scratch_arch_ok[dev] = (major == 10 && minor == 0);
-        if (!g_scratch_arch_ok[dev]) return MQ_ERR_ARCH;
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MQ_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return MQ_ERR_CUDA;
+    if (!(major == 10 && minor == 0)) return MQ_ERR_ARCH;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MQ_ERR_CUDA;
+    *addr = p;
     return MQ_OK;
 }
 
@@ -56,9 +49,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" int mq_linear_w4a4_noalloc(const void* x, int64_t M, int64_t K, const uint8_t* w_codes,
                                       const uint8_t* w_scales, const float* alpha_w, int64_t N, void* y,
                                       void* stream) {
-    // Every synchronous check comes before anything is enqueued.
+    // Every synchronous check of mq_linear_w4a4 comes before anything is
+    // enqueued (its shape limits too, so the size below cannot overflow).
     if (!x || !w_codes || !w_scales || !alpha_w || !y) return MQ_ERR_INVALID_ARG;
-    if (M <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return MQ_ERR_SHAPE;
+    const int shape = mq::check_linear_shape(M, N, K);
+    if (shape != MQ_OK) return shape;
     if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y)) return MQ_ERR_ALIGN;
     const size_t need = mq_linear_w4a4_workspace_bytes(M, K);
     if (need == 0) return MQ_ERR_SHAPE;

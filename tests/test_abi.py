@@ -85,3 +85,25 @@ def test_host_validation_without_gpu(libmq):
     assert libmq.mq_mlp_w4a4(p16, 128, 1024, p16, p16, p16, 64, p16, p16, p16, 64, p16, p16, 1 << 30, None) == -2
     assert libmq.mq_mlp_w4a4(p16, 128, 1024, None, p16, p16, 256, p16, p16, p16, 64, p16, p16, 1 << 30, None) == -1
     assert libmq.mq_status_string(-7) == b"MQ_ERR_TIMEOUT"
+
+
+def test_noalloc_constant_and_host_checks(libmq):
+    """The binding's scratch size is the header's, and the allocation-free
+    linear refuses bad shapes before it touches the device: the shape limits of
+    mq_linear_w4a4 come first, then the scratch size."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    text = open(os.path.join(HEADER_DIR, "mq.h")).read()
+    m = re.search(r"#define\s+MQ_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m, "MQ_NOALLOC_SCRATCH_BYTES not found in mq.h"
+    assert mq.MQ_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+    f = libmq.mq_linear_w4a4_noalloc
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    f.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp]
+    f.restype = ctypes.c_int
+    p16 = vp(4096)
+    assert f(p16, 128, 100, p16, p16, p16, 256, p16, None) == -2                 # K % 64
+    assert f(p16, 128, 1024, p16, p16, p16, (1 << 31) + 1, p16, None) == -2      # N beyond the row limit
+    assert f(p16, 1 << 40, 1 << 20, p16, p16, p16, 256, p16, None) == -2         # M * K beyond the 32-bit block index
+    assert f(None, 128, 1024, p16, p16, p16, 256, p16, None) == -1               # null
+    assert f(vp(4097), 128, 1024, p16, p16, p16, 256, p16, None) == -3           # misaligned
+    assert f(p16, 131072, 4096, p16, p16, p16, 256, p16, None) == -5             # beyond the scratch
