@@ -84,12 +84,13 @@ constexpr int MAX_STAGES = 10;
 constexpr int BARRIER_BYTES = 512;
 constexpr int SMEM_LIMIT = 232448;                  // dynamic shared memory per block on sm_100
 
-// PAIR: CTAs per output tile (1 or 2).  BK: K elements per pipeline stage
-// (128 or 256; the code tiles use the 64- or 128-byte swizzle).
-template <int PAIR, int BK>
+constexpr int BK = 256;                             // K elements per pipeline stage
+
+// PAIR: CTAs per output tile (1 or 2).
+template <int PAIR>
 struct Cfg {
     static constexpr int NKB = BK / MMA_K;                    // MMAs per stage
-    static constexpr int ROW_BYTES = BK / 2;                  // bytes of one code row per stage
+    static constexpr int ROW_BYTES = BK / 2;                  // bytes of one code row per stage (the 128-byte swizzle)
     static constexpr int A_BYTES = BM * ROW_BYTES;
     static constexpr int B_ROWS = BN / PAIR;                  // B rows staged by one CTA
     static constexpr int B_BYTES = B_ROWS * ROW_BYTES;
@@ -109,7 +110,7 @@ struct Cfg {
                                                             : (TMEM_STAGES < MAX_STAGES ? TMEM_STAGES : MAX_STAGES);
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*align*/ + BARRIER_BYTES;
     static constexpr int TILE_M = BM * PAIR;
-    static constexpr uint32_t SWIZZLE = ROW_BYTES == 128 ? 2 : 4;     // descriptor layout: 128B / 64B swizzle
+    static constexpr uint32_t SWIZZLE = 2;                            // descriptor layout: 128-byte swizzle
     static constexpr uint32_t SBO = 8 * ROW_BYTES;                    // 8-row swizzle atom
     // Instruction descriptor of kind::mxf4nvf4: E2M1 x E2M1, UE4M3 scales,
     // K-major A and B, M = TILE_M, N = 256, dense K = 64.
@@ -118,7 +119,7 @@ struct Cfg {
                                     | ((uint32_t)(BN >> 3) << 17)
                                     | (0u << 23)           // scale format UE4M3
                                     | ((uint32_t)(TILE_M >> 4) << 24);
-    static_assert(BK == 128 || BK == 256, "stage depth");
+    static_assert(NKB == 4 && ROW_BYTES == 128, "stage depth: four MMAs, 128-byte code rows");
     static_assert(STAGES >= 2 && STAGES <= MAX_STAGES, "stage count");
     static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM budget");
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the swizzle atoms");
@@ -136,11 +137,9 @@ struct Params {
     int* status;
     long long timeout;
     int fault_skip_first_load;
-    int y_tma;               // Y is written by TMA stores (tmap_y is valid)
+    int y_tma;               // pair form: Y is written by TMA stores (tmap_y is valid; needs N % 8 == 0)
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
     int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
-    int sfb_tma;             // B's two scale slices of a stage arrive as one TMA box (tmap_sfb is valid)
-    int sfa_tma;             // A's scale slice of a stage arrives as a TMA box (tmap_sfa is valid)
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
     uint8_t* x_codes;        // fused linear: where A's codes are written
     uint8_t* x_scales;       // fused linear: where A's scales are written
@@ -256,12 +255,12 @@ __device__ __forceinline__ void commit_to_all(uint64_t* bar) {
     else mma_commit(bar);
 }
 
-template <int PAIR, int BK, bool QUANT, bool SWIGLU>
+template <int PAIR, bool QUANT, bool SWIGLU>
 __global__ void __launch_bounds__(THREADS, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
        const __grid_constant__ CUtensorMap tmap_y, const __grid_constant__ CUtensorMap tmap_sfb,
        const __grid_constant__ CUtensorMap tmap_sfa, Params p) {
-    using C = Cfg<PAIR, BK>;
+    using C = Cfg<PAIR>;
     constexpr int NKB = C::NKB;
     constexpr int A_BYTES = C::A_BYTES;
     constexpr int SFA_BYTES = C::SFA_BYTES;
@@ -301,8 +300,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         prefetch_tmap(&tmap_a);
         prefetch_tmap(&tmap_b);
         if (C::TMA_STORE && p.y_tma) prefetch_tmap(&tmap_y);
-        if (p.sfb_tma) prefetch_tmap(&tmap_sfb);
-        if (p.sfa_tma) prefetch_tmap(&tmap_sfa);
+        prefetch_tmap(&tmap_sfb);
+        prefetch_tmap(&tmap_sfa);
     }
     if (warp == 1) {
         if (PAIR == 2) {
@@ -346,8 +345,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         break;
                     }
                     pending &= ~(1u << st);
-                    const int nkb = min(NKB, p.kblocks - kt * NKB);
-                    const uint32_t sf_bytes = nkb * 512;               // one 128-row scale slice
                     if (skip) {     // failure-detection test hook: never complete this stage
                         skip = false;
                     } else {
@@ -367,24 +364,16 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             tma_load_2d(stage_b(st), &tmap_b, &s->ready[st], kt * C::ROW_BYTES, brow);
                             if (!QUANT) tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
                         }
-                        if (SWIGLU) {
-                            // the gate and the up scale slices in one box of a 3-D view
-                            mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + (p.sfa_tma ? SFB_BYTES / 2 : sf_bytes));
+                        // the scale slices: B's two 128-row slices in one box
+                        // (rows nb*2, nb*2+1 of the [row tile][k atom] array;
+                        // SwiGLU form: the gate slice and the matching up
+                        // slice in one box of a 3-D view), then A's slice; the
+                        // boxes always land whole, zero past the ends
+                        mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + SFA_BYTES);
+                        if (SWIGLU)
                             tma_load_3d(stage_sfb(st), &tmap_sfb, &s->sf_full[st], (int)(ka * 64), nb, 0);
-                        } else if (p.sfb_tma) {
-                            // B's two 128-row scale slices in one box (rows
-                            // nb*2, nb*2+1 of the [row tile][k atom] array);
-                            // the box always lands whole, zero past the ends
-                            mbar_arrive_expect_tx(&s->sf_full[st], SFB_BYTES + (p.sfa_tma ? SFB_BYTES / 2 : sf_bytes));
+                        else
                             tma_load_2d(stage_sfb(st), &tmap_sfb, &s->sf_full[st], (int)(ka * 64), nb * 2);
-                        } else {
-                            mbar_arrive_expect_tx(&s->sf_full[st], 2 * sf_bytes + (p.sfa_tma ? SFB_BYTES / 2 : sf_bytes));
-                            for (int rt = 0; rt < 2; ++rt) {
-                                const int64_t bt = min(nb * 2 + rt, p.b_row_tiles - 1);
-                                bulk_load(stage_sfb(st) + rt * (SFB_BYTES / 2),
-                                          p.b_scales + (bt * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
-                            }
-                        }
                         if (QUANT && arow / 128 < p.a_row_tiles) {
                             // A's block (arow, kt) is written by quantizer warps (of any CTA)
                             const int* f = p.flags + (int64_t)(arow / 128) * p.k_stages + kt;
@@ -396,10 +385,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                             }
                             fence_proxy_async_global();
                         }
-                        if (p.sfa_tma)
-                            tma_load_2d(stage_sfa(st), &tmap_sfa, &s->sf_full[st], (int)(ka * 64), (int)at);
-                        else
-                            bulk_load(stage_sfa(st), p.a_scales + (at * p.katoms + ka) * 512, sf_bytes, &s->sf_full[st]);
+                        tma_load_2d(stage_sfa(st), &tmap_sfa, &s->sf_full[st], (int)(ka * 64), (int)at);
                         if (QUANT) {
                             if (PAIR == 2) tma_load_2d_pair(stage_a(st), &tmap_a, bar0, kt * C::ROW_BYTES, arow);
                             else tma_load_2d(stage_a(st), &tmap_a, &s->ready[st], kt * C::ROW_BYTES, arow);
@@ -436,49 +422,43 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     break;
                 }
                 tc_fence_after();
-                // The tensor pipe queues about one MMA behind the running one,
-                // so the gap between the last MMA of a stage and the first of
-                // the next must stay short: the wait for the next stage's
-                // barrier is taken while the stage's last MMAs are still queued.
-                bool ok = mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag);
-                tc_fence_after();
-                for (int kt = 0; ok && kt < p.k_stages; ++kt) {
-                    // the stage's codes are in shared memory and its scales in TMEM
+                // Per stage: wait for the stage (its codes in shared memory,
+                // its scales in TMEM), then its MMAs back to back, then the
+                // commit that frees the stage.  Any other instruction between
+                // two MMAs -- even a branch not taken, let alone a barrier
+                // poll -- costs the tensor pipe ~30-60 cycles per MMA (clock64
+                // traces: 773 SM cycles per 4-MMA stage with the next stage's
+                // wait placed before the last MMA, 700 with this order, 512
+                // back to back), so the waits sit only at stage boundaries.
+                bool ok = true;
+                for (int kt = 0; kt < p.k_stages; ++kt) {
+                    if (!mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
                     const int nkb = min(NKB, p.kblocks - kt * NKB);
-                    const int nst = st + 1 == p.stages ? 0 : st + 1;
-                    const uint32_t nphase = st + 1 == p.stages ? phase ^ 1 : phase;
-                    const bool more = kt + 1 < p.k_stages;
-                    // descriptors of the stage's first K step; the next steps
-                    // start MMA_K / 2 bytes further (address field in 16-byte units)
                     const uint64_t ad0 = smem_desc(smem_u32(stage_a(st)), 16, C::SBO, C::SWIZZLE);
                     const uint64_t bd0 = smem_desc(smem_u32(stage_b(st)), 16, C::SBO, C::SWIZZLE);
                     const uint32_t sf = tmem + SF_COL + st * SF_COLS_PER_STAGE;
-                    auto mma = [&](int kb) {
+                    const uint32_t acc0 = kt != 0;
+                    auto mma = [&](int kb, uint32_t acc) {
                         const uint64_t step = (uint64_t)(kb * (MMA_K / 2) >> 4);
                         if (PAIR == 2)
                             mma_mxf4nvf4_pair(tmem + ACC_COL, ad0 + step, bd0 + step, C::IDESC, sf + kb * 4,
-                                              sf + SFB_OFF + kb * 8, (kt | kb) != 0);
+                                              sf + SFB_OFF + kb * 8, acc);
                         else
                             mma_mxf4nvf4(tmem + ACC_COL, ad0 + step, bd0 + step, C::IDESC, sf + kb * 4,
-                                         sf + SFB_OFF + kb * 8, (kt | kb) != 0);
+                                         sf + SFB_OFF + kb * 8, acc);
                     };
-                    bool next_ok = true;
                     if (nkb == NKB) {
-                        // a full stage: no branch between two MMAs (one measured
-                        // ~30% lower tensor-pipe throughput)
+                        // a full stage: straight-line code from the first MMA to the last
+                        mma(0, acc0);
 #pragma unroll
-                        for (int kb = 0; kb < NKB - 1; ++kb) mma(kb);
-                        if (more) next_ok = mbar_wait_bounded(&s->ready[nst], nphase, p.timeout, abort_flag);
-                        mma(NKB - 1);
+                        for (int kb = 1; kb < NKB; ++kb) mma(kb, 1u);
                     } else {
-                        for (int kb = 0; kb < nkb; ++kb) mma(kb);
-                        if (more) next_ok = mbar_wait_bounded(&s->ready[nst], nphase, p.timeout, abort_flag);
+                        for (int kb = 0; kb < nkb; ++kb) mma(kb, (kt | kb) != 0);
                     }
                     commit_to_all<PAIR>(&s->empty[st]);
-                    st = nst;
-                    phase = nphase;
-                    if (!next_ok) ok = false;
-                    tc_fence_after();
+                    st = st + 1 == p.stages ? 0 : st + 1;
+                    phase = st == 0 ? phase ^ 1 : phase;
                 }
                 if (!ok) {
                     raise_abort(s, p);
@@ -576,7 +556,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 // The stage's 12 NKB scale columns are contiguous in TMEM: A's
                 // (4 per MMA), then B's (8 per MMA).  All shared-memory reads
                 // first, then one store per operand.  In a K-tail stage the
-                // columns past the last MMA get stale bytes that nothing reads.
+                // columns past the last MMA get the boxes' zero fill, which
+                // nothing reads.
                 uint32_t va[4 * NKB], vb[8 * NKB];
 #pragma unroll
                 for (int kb = 0; kb < NKB; ++kb) {
@@ -587,13 +568,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     vb[8 * kb] = b0.x; vb[8 * kb + 1] = b0.y; vb[8 * kb + 2] = b0.z; vb[8 * kb + 3] = b0.w;
                     vb[8 * kb + 4] = b1.x; vb[8 * kb + 5] = b1.y; vb[8 * kb + 6] = b1.z; vb[8 * kb + 7] = b1.w;
                 }
-                if constexpr (NKB == 4) {
-                    tmem_st_32x32b_x16(t, va);
-                    tmem_st_32x32b_x32(t + SFB_OFF, vb);
-                } else {
-                    tmem_st_32x32b_x8(t, va);
-                    tmem_st_32x32b_x16(t + SFB_OFF, vb);
-                }
+                tmem_st_32x32b_x16(t, va);
+                tmem_st_32x32b_x32(t + SFB_OFF, vb);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -922,16 +898,16 @@ struct FormState {
     bool attr_set = false;
     int max_units = 0;      // co-resident CTAs (PAIR 1) or clusters (PAIR 2)
 };
-FormState g_form[64][3][2][2][2];
+FormState g_form[64][3][2][2];
 
-template <int PAIR, int BK, bool QUANT, bool SWIGLU = false>
+template <int PAIR, bool QUANT, bool SWIGLU = false>
 cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     using namespace gemm;
-    using C = Cfg<PAIR, BK>;
+    using C = Cfg<PAIR>;
     int dev = 0;
     cudaGetDevice(&dev);
-    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][BK == 256][QUANT][SWIGLU];
-    auto kernel = k_gemm<PAIR, BK, QUANT, SWIGLU>;
+    FormState& fs = g_form[dev < 64 ? dev : 63][PAIR][QUANT][SWIGLU];
+    auto kernel = k_gemm<PAIR, QUANT, SWIGLU>;
     if (!fs.attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
@@ -961,23 +937,21 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     memset(&my, 0, sizeof(my));
     memset(&msfb, 0, sizeof(msfb));
+    memset(&msfa, 0, sizeof(msfa));
     // the SwiGLU form writes H [M, inter] (inter = N / 2) by TMA stores
     const int64_t n_out = SWIGLU ? a.swiglu_inter : a.N;
-    const int y_mode = SWIGLU ? 1 : env_int("MQ_GEMM_YTMA", 0, 1, 1);
-    const bool y_tma = C::TMA_STORE && y_mode != 0 && make_y_map(&my, a.y, a.M, n_out);
-    bool sfb_tma;
+    // pair form: Y by TMA stores when its rows are 16-byte multiples, else
+    // the element stores of the ragged path
+    const bool y_tma = C::TMA_STORE && make_y_map(&my, a.y, a.M, n_out);
     if (SWIGLU) {
         if (!y_tma || a.N != 2 * a.swiglu_inter || !a.h_amax ||
             !make_gate_up_scale_map(&msfb, a.b_scales, a.swiglu_inter, scale_atom_cols(a.K), C::NKB))
             return cudaErrorInvalidValue;
-        sfb_tma = true;
-    } else {
-        sfb_tma = env_int("MQ_GEMM_SFB_TMA", 0, 1, 1) &&
-                  make_scale_map(&msfb, a.b_scales, padded_rows(a.N) / 128, scale_atom_cols(a.K), 2, C::NKB);
+    } else if (!make_scale_map(&msfb, a.b_scales, padded_rows(a.N) / 128, scale_atom_cols(a.K), 2, C::NKB)) {
+        return cudaErrorInvalidValue;
     }
-    memset(&msfa, 0, sizeof(msfa));
-    const bool sfa_tma = env_int("MQ_GEMM_SFA_TMA", 0, 1, 1) &&
-                         make_scale_map(&msfa, a.a_scales, padded_rows(a.M) / 128, scale_atom_cols(a.K), 1, C::NKB);
+    if (!make_scale_map(&msfa, a.a_scales, padded_rows(a.M) / 128, scale_atom_cols(a.K), 1, C::NKB))
+        return cudaErrorInvalidValue;
     Params p{};
     p.a_scales = a.a_scales;
     p.b_scales = a.b_scales;
@@ -1000,9 +974,7 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.status = a.status;
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
-    p.y_tma = y_tma ? y_mode : 0;
-    p.sfb_tma = sfb_tma ? 1 : 0;
-    p.sfa_tma = sfa_tma ? 1 : 0;
+    p.y_tma = y_tma ? 1 : 0;
     p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
     p.stages = env_int("MQ_GEMM_STAGES", 2, C::STAGES, C::STAGES);
     p.x = static_cast<const uint16_t*>(a.x);
@@ -1048,31 +1020,24 @@ int env_choice(const char* name, int a, int b, int dflt) {
 }  // namespace
 
 int64_t fused_flag_count(int64_t M, int64_t K) {
-    using C = gemm::Cfg<2, 256>;
+    using C = gemm::Cfg<2>;
     return padded_rows(M) / 128 * ((K / gemm::MMA_K + C::NKB - 1) / C::NKB);
 }
 
-// The 2-CTA form for M > 128, the 1-CTA form otherwise.  MQ_GEMM_FORM=1|2 and
-// MQ_GEMM_BK=128|256 force a variant (the tests check every variant on the
-// same shapes); the fused linear always runs with 256-element K stages.
+// The 2-CTA form for M > 128, the 1-CTA form otherwise; the decode form for
+// M <= 64 (unfused).  MQ_GEMM_FORM=1|2 forces the prefill form and
+// MQ_GEMM_DECODE=0 keeps small M on the prefill kernel (the tests compare
+// the forms on the same shapes).
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
-    if (a.swiglu_inter > 0) return launch_form<2, 256, false, true>(a, num_sms, stream);
-    // few rows of A (decode-shaped): the weight-streaming split-K form,
-    // unless MQ_GEMM_DECODE=0 or a variant is forced
+    if (a.swiglu_inter > 0) return launch_form<2, false, true>(a, num_sms, stream);
     const char* dv = getenv("MQ_GEMM_DECODE");
     if (!(dv && dv[0] == '0') && !getenv("MQ_GEMM_FORM") && !a.x && a.M <= 64) {
         const cudaError_t e = launch_gemm_decode(a, num_sms, stream);
         if (e != cudaErrorNotSupported) return e;
     }
     const int form = env_choice("MQ_GEMM_FORM", 1, 2, a.M > gemm::BM ? 2 : 1);
-    if (a.x) return form == 2 ? launch_form<2, 256, true>(a, num_sms, stream)
-                              : launch_form<1, 256, true>(a, num_sms, stream);
-    const int bk = env_choice("MQ_GEMM_BK", 128, 256, 256);
-    if (form == 2)
-        return bk == 128 ? launch_form<2, 128, false>(a, num_sms, stream)
-                         : launch_form<2, 256, false>(a, num_sms, stream);
-    return bk == 128 ? launch_form<1, 128, false>(a, num_sms, stream)
-                     : launch_form<1, 256, false>(a, num_sms, stream);
+    if (a.x) return form == 2 ? launch_form<2, true>(a, num_sms, stream) : launch_form<1, true>(a, num_sms, stream);
+    return form == 2 ? launch_form<2, false>(a, num_sms, stream) : launch_form<1, false>(a, num_sms, stream);
 }
 
 }  // namespace mq

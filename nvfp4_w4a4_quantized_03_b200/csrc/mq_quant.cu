@@ -1,13 +1,17 @@
 // mq_quant.cu -- the two HBM-bound passes of NVFP4 quantization.
 //
-//   k_amax      : amax = max |x| over a bf16 tensor, then the tensor-level
-//                 scale alpha_x = fl32(amax / (q_max * 448)) = fl32(amax / 2688)
-//                 (alpha_x = 1 for an all-zero tensor).
-//   k_quantize  : per 16-element block along K,
-//                   sigma_b = Pi_E4M3(fl32(amax_b / fl32(6 alpha_x)))
-//                   q_i     = Pi_E2M1(fl32(x_i * fl32(1 / fl32(alpha_x sigma_b))))
-//                 codes packed two per byte (lower K index in the low nibble),
-//                 scales written straight into the block-scaled MMA's layout.
+//   k_amax                : amax = max |x| over a bf16 tensor, then the
+//                           tensor-level scale alpha_x = fl32(amax / (q_max * 448))
+//                           = fl32(amax / 2688) (alpha_x = 1 for an all-zero tensor).
+//   k_quantize_ws         : per 16-element block along K,
+//                             sigma_b = Pi_E4M3(fl32(amax_b / fl32(6 alpha_x)))
+//                             q_i     = Pi_E2M1(fl32(x_i * fl32(1 / fl32(alpha_x sigma_b))))
+//                           codes packed two per byte (lower K index in the low
+//                           nibble), scales written straight into the block-scaled
+//                           MMA's layout.
+//   k_quantize_onepass_ws : both in one cooperative launch (amax pass, grid
+//                           barrier, quantization pass over the data the amax
+//                           pass left in L2), for the linear.
 //
 // The formulas are NVFP4's two-level microscaling as given in
 // "Mix-Quant：面向智能体LLM的量化预填充与精确解码" (paper.rainbus.top digest),
@@ -110,8 +114,6 @@ k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ t
     }
 }
 
-constexpr int QUANT_THREADS = 256;
-
 // Quantizes the four consecutive 16-element blocks [4q, 4q + 4) of row `row`:
 // 128 bytes of x in, 32 code bytes and one 32-bit scale word (the four block
 // scales, one word of the MMA layout) out.  Padding rows (row >= rows) get a
@@ -120,9 +122,9 @@ constexpr int QUANT_THREADS = 256;
 // sector per request instead of two half-sector writes, which took the
 // stand-alone quantizer on 8192 x 12288 from 51 to 45 us (the threads of a
 // warp write 32 different rows, so no two stores of a warp share a sector).
-__device__ __forceinline__ void quantize_quad(const uint4* __restrict__ x, int64_t rows, int64_t K, uint32_t row,
-                                              uint32_t q, float alpha, uint4* __restrict__ codes,
-                                              uint8_t* __restrict__ scales, const uint4 (&v)[8]) {
+__device__ __forceinline__ void quantize_quad(int64_t rows, int64_t K, uint32_t row, uint32_t q, float alpha,
+                                              uint4* __restrict__ codes, uint8_t* __restrict__ scales,
+                                              const uint4 (&v)[8]) {
     uint32_t word = 0;
     if (row < rows) {
         uint32_t c[8];
@@ -140,201 +142,27 @@ __device__ __forceinline__ void quantize_quad(const uint4* __restrict__ x, int64
     *reinterpret_cast<uint32_t*>(scales + scale_byte_offset(row, 4 * (int64_t)q, K / 64)) = word;
 }
 
-__device__ __forceinline__ void load_quad(const uint4* __restrict__ x, int64_t rows, int64_t K, uint32_t row,
-                                          uint32_t q, uint4 (&v)[8]) {
-    if (row < rows) {
-        const uint4* src = x + ((int64_t)row * (K / 64) + q) * 8;      // 128 bytes per quad
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = src[j];
-    }
-}
-
-// One thread per four consecutive blocks of a row (K is a multiple of 64);
-// threads run over the padded row range so the padding rows of the scale
-// buffer are written as zeros.
-__global__ void __launch_bounds__(QUANT_THREADS)
-k_quantize(const uint4* __restrict__ x, int64_t rows, int64_t prows, int64_t K,
-           const float* __restrict__ alpha_p, uint4* __restrict__ codes, uint8_t* __restrict__ scales) {
-    const uint32_t quads = (uint32_t)(K / 64);
-    const int64_t g = (int64_t)blockIdx.x * QUANT_THREADS + threadIdx.x;
-    if (g >= prows * quads) return;
-    const uint32_t row = (uint32_t)g / quads, q = (uint32_t)g - row * quads;
-    uint4 v[8];
-    load_quad(x, rows, K, row, q, v);
-    quantize_quad(x, rows, K, row, q, __ldg(alpha_p), codes, scales, v);
-}
-
 // ---------------------------------------------------------------------------
-// k_quantize_tiles: the same quantization with X brought into shared memory
-// by TMA, 256 rows x 64 elements (32 KB) per box in the 128-byte swizzle.
-// Thread t quantizes row t of a box (four blocks, one scale word) from its
-// 128-byte row of the box; the swizzle puts the 16-byte chunk j of row t at
-// chunk j ^ (t % 8), so the eight 16-byte shared-memory reads of a warp are
-// conflict-free.  A ring of QT_STAGES boxes per CTA keeps the loads in
-// flight while the previous box is quantized.  (Loading the same data with
-// eight 16-byte global loads per thread measured the L1 at 90% of its
-// throughput: every warp-wide load touched 32 cache lines.)
+// The quantizers stream X through shared memory by TMA, 256 rows x 64
+// elements (32 KB) per box in the 128-byte swizzle.  Thread t quantizes row t
+// of a box (four blocks, one scale word) from its 128-byte row of the box;
+// the swizzle puts the 16-byte chunk j of row t at chunk j ^ (t % 8), so the
+// eight 16-byte shared-memory reads of a warp are conflict-free.  A ring of
+// QT_STAGES boxes per block keeps the loads in flight while earlier boxes are
+// quantized.  (Loading the same data with eight 16-byte global loads per
+// thread measured the L1 at 90% of its throughput, every warp-wide load
+// touching 32 cache lines, and ran 17-23% slower.)
 constexpr int QT_THREADS = 256;
 constexpr int QT_ROWS = 256;
 constexpr int QT_STAGES = 3;
 constexpr int QT_BOX_BYTES = QT_ROWS * 128;
 constexpr int QT_SMEM = QT_STAGES * QT_BOX_BYTES + 1024;
 
-__global__ void __launch_bounds__(QT_THREADS, 2)
-k_quantize_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
-                 const float* __restrict__ alpha_p, uint4* __restrict__ codes, uint8_t* __restrict__ scales) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[QT_STAGES];
-    const int64_t kgroups = K / 64;
-    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < QT_STAGES; ++i) mbar_init(&full[i], 1);
-        fence_mbar_init();
-        prefetch_tmap(&xmap);
-    }
-    __syncthreads();
-    pdl_launch_dependents();
-    pdl_wait();
-    auto issue = [&](int64_t t, int st) {
-        mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
-        tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
-                    (int32_t)(t / kgroups) * QT_ROWS);
-    };
-    if (threadIdx.x == 0)
-        for (int i = 0; i < QT_STAGES; ++i)
-            if (blockIdx.x + (int64_t)i * gridDim.x < ntiles) issue(blockIdx.x + (int64_t)i * gridDim.x, i);
-    const float alpha = __ldg(alpha_p);
-    int it = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-        const int st = it % QT_STAGES;
-        // the box's bytes landed (bounded: a copy that never lands ends the
-        // block rather than hanging it)
-        if (!mbar_wait_bounded(&full[st], (uint32_t)(it / QT_STAGES) & 1, 4000000000LL, nullptr)) break;
-        const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
-        const uint32_t kg = (uint32_t)(t % kgroups);
-        if (row < prows) {
-            const uint8_t* src = base + st * QT_BOX_BYTES + threadIdx.x * 128;
-            uint4 v[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
-            quantize_quad(nullptr, rows, K, (uint32_t)row, kg, alpha, codes, scales, v);
-        }
-        fence_proxy_async_shared();   // the reads are performed before the slot's next TMA load
-        __syncthreads();     // every thread is done with this box
-        if (threadIdx.x == 0 && t + (int64_t)QT_STAGES * gridDim.x < ntiles) issue(t + (int64_t)QT_STAGES * gridDim.x, st);
-    }
-}
-
 // ---------------------------------------------------------------------------
-// k_quantize_onepass_tiles: alpha_x and the codes/scales of X in one
-// cooperative launch, X streamed through the same TMA ring of 256 x 64
-// boxes as k_quantize_tiles.  Each block takes the boxes t = block, block +
-// grid, ... ; "items" 0..n-1 are those boxes in order (phase 1: max |x|),
-// items n..2n-1 the same boxes in reverse order (phase 2: quantize), so the
-// boxes read last in phase 1 (the likeliest to be in L2) are read first in
-// phase 2, and the first boxes of phase 2 are already in flight while the
-// grid barrier between the phases completes.  Rows past the end arrive as
-// zeros, which leave the max unchanged.
-__global__ void __launch_bounds__(QT_THREADS, 2)
-k_quantize_onepass_tiles(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
-                         uint32_t* __restrict__ ws, float* __restrict__ alpha_out, uint4* __restrict__ codes,
-                         uint8_t* __restrict__ scales, int* __restrict__ status, long long timeout) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[QT_STAGES];
-    __shared__ uint32_t red[QT_THREADS / 32];
-    __shared__ int ok_shared;
-    __shared__ float alpha_shared;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    pdl_launch_dependents();
-    pdl_wait();
-    const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(&ws[WS_GENERATION]);
-    const int64_t kgroups = K / 64;
-    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * kgroups;
-    const int64_t n = ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;   // boxes of this block
-    auto box_of = [&](int64_t item) -> int64_t {   // item -> box index
-        const int64_t i = item < n ? item : 2 * n - 1 - item;
-        return blockIdx.x + i * gridDim.x;
-    };
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < QT_STAGES; ++i) mbar_init(&full[i], 1);
-        fence_mbar_init();
-        prefetch_tmap(&xmap);
-        ok_shared = 1;
-    }
-    __syncthreads();
-    auto issue = [&](int64_t item) {
-        const int64_t t = box_of(item);
-        const int st = (int)(item % QT_STAGES);
-        mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
-        tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
-                    (int32_t)(t / kgroups) * QT_ROWS);
-    };
-    if (threadIdx.x == 0)
-        for (int64_t i = 0; i < QT_STAGES && i < 2 * n; ++i) issue(i);
-    uint32_t m = 0;
-    float alpha = 0.0f;
-    // end of phase 1: fold this block's max, then the grid barrier (every
-    // block takes part, also one without boxes)
-    auto finish_phase1 = [&]() {
-        uint32_t v = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
-        if (lane == 0) red[warp] = v;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t w = 0;
-            for (int k = 0; k < QT_THREADS / 32; ++k) w = max(w, red[k]);
-            if (!amax_grid_barrier(ws, w, gen0, alpha_out, timeout)) {
-                ok_shared = 0;
-                if (status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
-            }
-            alpha_shared = *reinterpret_cast<volatile float*>(alpha_out);
-        }
-        __syncthreads();
-        alpha = alpha_shared;
-    };
-    if (n == 0) finish_phase1();
-    for (int64_t item = 0; item < 2 * n; ++item) {
-        if (item == n) finish_phase1();
-        const int st = (int)(item % QT_STAGES);
-        // a box that never lands, or a timed-out barrier, ends the block once
-        // its copies in flight have landed (they are waited for below)
-        const bool landed = mbar_wait_bounded(&full[st], (uint32_t)(item / QT_STAGES) & 1, timeout, nullptr);
-        if (!__syncthreads_and(landed && ok_shared)) {     // the same decision in every thread
-            if (threadIdx.x == 0 && status) atomicExch(status, -7);
-            ok_shared = 0;
-            break;
-        }
-        const uint8_t* src = base + st * QT_BOX_BYTES + threadIdx.x * 128;
-        uint4 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (threadIdx.x & 7)) << 4));
-        if (item < n) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) m = absmax_vec(m, v[j]);
-        } else {
-            const int64_t t = box_of(item);
-            const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
-            if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
-        }
-        fence_proxy_async_shared();   // the reads are performed before the slot's next TMA load
-        __syncthreads();     // every thread is done with this box
-        if (threadIdx.x == 0 && item + QT_STAGES < 2 * n) issue(item + QT_STAGES);
-    }
-    // copies still in flight after an early exit land before the block ends
-    if (threadIdx.x == 0 && !ok_shared) {
-        const long long t0 = clock64();
-        while (clock64() - t0 < 200000) {
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// k_quantize_ws: k_quantize_tiles as a producer/consumer pipeline (one lane
-// of warp 8 streams this block's boxes into the ring as slots free up; warps
-// 0..7 quantize one box row per thread and release a slot with one arrival
-// per warp).  Before a warp releases a slot, each of its threads executes a
+// k_quantize_ws: a producer/consumer pipeline (one lane of warp 8 streams
+// this block's boxes into the ring as slots free up; warps 0..7 quantize one
+// box row per thread and release a slot with one arrival per warp, so no
+// warp waits for the slowest one of the block between boxes).  Before a warp releases a slot, each of its threads executes a
 // generic-to-async proxy fence: the mbarrier's release/acquire alone does not
 // order the threads' shared-memory reads before the next TMA write into the
 // slot, and without the fence rows were seen quantized from the next box.
@@ -396,7 +224,7 @@ k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t pr
         if (lane == 0) mbar_arrive(&empty[st]);       // this warp is done with the slot
         const int64_t t = blockIdx.x + i * gridDim.x;
         const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
-        if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
+        if (row < prows) quantize_quad(rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
     }
 }
 
@@ -510,147 +338,45 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
         } else {
             const int64_t t = box_of(item);
             const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
-            if (row < prows) quantize_quad(nullptr, rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
+            if (row < prows) quantize_quad(rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
         }
-    }
-}
-
-constexpr int ONEPASS_THREADS = 256;
-
-// alpha_x and the codes/scales of a [rows, K] tensor in one launch.  Every
-// block is resident (cooperative launch).
-//   phase 1: max |x| over the whole tensor (eight 16-byte loads in flight per
-//            thread); blocks fold their max into ws with one atomic; the last
-//            block computes alpha_x, resets the counters and bumps the
-//            generation word, which releases all blocks (bounded spin).
-//   phase 2: one 16-element block per thread and step, walking the tensor
-//            from its end so the most recently read lines (still in L2) are
-//            quantized first.
-__global__ void __launch_bounds__(ONEPASS_THREADS, 4)
-k_quantize_onepass(const uint4* __restrict__ x, int64_t rows, int64_t prows, int64_t K,
-                   uint32_t* __restrict__ ws, float* __restrict__ alpha_out, uint4* __restrict__ codes,
-                   uint8_t* __restrict__ scales, int* __restrict__ status, long long timeout) {
-    __shared__ uint32_t red[ONEPASS_THREADS / 32];
-    __shared__ bool ok_shared;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const uint32_t gen0 = *reinterpret_cast<volatile uint32_t*>(&ws[WS_GENERATION]);
-
-    // ---- phase 1: amax
-    const int64_t nvec = rows * K / 8;
-    const int64_t stride = (int64_t)gridDim.x * ONEPASS_THREADS;
-    int64_t i = (int64_t)blockIdx.x * ONEPASS_THREADS + threadIdx.x;
-    uint32_t m = 0;
-    for (; i < nvec; i += 8 * stride) {
-        uint4 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = x[min(i + j * stride, nvec - 1)];   // a repeat leaves the max unchanged
-#pragma unroll
-        for (int j = 0; j < 8; ++j) m = absmax_vec(m, v[j]);
-    }
-    uint32_t v = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t w = 0;
-        for (int k = 0; k < ONEPASS_THREADS / 32; ++k) w = max(w, red[k]);
-        const bool ok = amax_grid_barrier(ws, w, gen0, alpha_out, timeout);
-        if (!ok && status) atomicExch(status, -7 /* MQ_ERR_TIMEOUT */);
-        ok_shared = ok;
-    }
-    __syncthreads();
-    if (!ok_shared) return;
-    const float alpha = *reinterpret_cast<volatile float*>(alpha_out);
-
-    // ---- phase 2: quantize, from the end of the tensor backwards (the
-    // lines phase 1 read last are the likeliest to still be in L2); one
-    // thread per four consecutive blocks of a row and step
-    const uint32_t quads = (uint32_t)(K / 64);
-    const int64_t total = prows * quads;                   // padded rows: their scales are zero
-    const int64_t steps = (total + stride - 1) / stride;
-    const int64_t t0 = (int64_t)blockIdx.x * ONEPASS_THREADS + threadIdx.x;
-    for (int64_t s = steps - 1; s >= 0; --s) {
-        const int64_t g = s * stride + t0;
-        if (g >= total) continue;
-        const uint32_t row = (uint32_t)g / quads, q = (uint32_t)g - row * quads;
-        uint4 v[8];
-        load_quad(x, rows, K, row, q, v);
-        quantize_quad(x, rows, K, row, q, alpha, codes, scales, v);
     }
 }
 
 cudaError_t launch_quantize_onepass(const void* x, int64_t rows, int64_t K, uint32_t* ws_words, float* alpha_out,
                                     uint8_t* codes, uint8_t* scales, int* status, long long timeout_cycles,
                                     cudaStream_t stream) {
-    static int blocks_per_sm[64] = {};
+    static int per_sm[64] = {};
     static int sms[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     const int d = dev < 64 ? dev : 63;
-    if (!blocks_per_sm[d]) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm[d], k_quantize_onepass,
-                                                                      ONEPASS_THREADS, 0);
-        if (e != cudaSuccess || blocks_per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+    if (!per_sm[d]) {
+        cudaError_t e = cudaFuncSetAttribute(k_quantize_onepass_ws, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             QT_SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[d], k_quantize_onepass_ws, QW_THREADS, QT_SMEM);
+        if (e != cudaSuccess || per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
         cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
     }
-    const int64_t prows = padded_rows(rows);
-    // the TMA-streamed form (MQ_ONEPASS_TILES=0 selects the per-thread-load form)
-    const char* tv = getenv("MQ_ONEPASS_TILES");
     CUtensorMap xmap;
-    if (!(tv && tv[0] == '0') && make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) {
-        static int tiles_per_sm[64] = {};
-        if (!tiles_per_sm[d]) {
-            cudaError_t e = cudaFuncSetAttribute(k_quantize_onepass_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 QT_SMEM);
-            if (e != cudaSuccess) return e;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&tiles_per_sm[d], k_quantize_onepass_tiles, QT_THREADS,
-                                                              QT_SMEM);
-            if (e != cudaSuccess || tiles_per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-        }
-        // every block resident (grid barrier) and every block owning at least one box
-        const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        cfg.dynamicSmemBytes = QT_SMEM;
-        cfg.stream = stream;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const char* wv = getenv("MQ_ONEPASS_WS");
-        if (!(wv && wv[0] == '0')) {
-            // the producer/consumer form (MQ_ONEPASS_WS=0: the block-synchronous ring)
-            static int ws_per_sm[64] = {};
-            if (!ws_per_sm[d]) {
-                cudaError_t e = cudaFuncSetAttribute(k_quantize_onepass_ws, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     QT_SMEM);
-                if (e != cudaSuccess) return e;
-                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ws_per_sm[d], k_quantize_onepass_ws, QW_THREADS,
-                                                                  QT_SMEM);
-                if (e != cudaSuccess || ws_per_sm[d] <= 0) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-            }
-            cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * ws_per_sm[d])));
-            cfg.blockDim = dim3(QW_THREADS);
-            return cudaLaunchKernelEx(&cfg, k_quantize_onepass_ws, xmap, rows, prows, K, ws_words, alpha_out,
-                                      reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
-        }
-        cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * tiles_per_sm[d])));
-        cfg.blockDim = dim3(QT_THREADS);
-        return cudaLaunchKernelEx(&cfg, k_quantize_onepass_tiles, xmap, rows, prows, K, ws_words, alpha_out,
-                                  reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
-    }
-    const int64_t need = (prows * (K / 64) + ONEPASS_THREADS - 1) / ONEPASS_THREADS;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)sms[d] * blocks_per_sm[d]));
+    if (!make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) return cudaErrorInvalidValue;
+    const int64_t prows = padded_rows(rows);
+    // every block resident (the grid barrier needs it: a cooperative launch
+    // guarantees it or refuses) and every block owning at least one box
+    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;     // all blocks resident: the grid barrier needs it
+    attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(ONEPASS_THREADS);
+    cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms[d] * per_sm[d])));
+    cfg.blockDim = dim3(QW_THREADS);
+    cfg.dynamicSmemBytes = QT_SMEM;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_quantize_onepass, reinterpret_cast<const uint4*>(x), rows, prows, K, ws_words,
-                              alpha_out, reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
+    return cudaLaunchKernelEx(&cfg, k_quantize_onepass_ws, xmap, rows, prows, K, ws_words, alpha_out,
+                              reinterpret_cast<uint4*>(codes), scales, status, timeout_cycles);
 }
 
 cudaError_t launch_amax(const void* x, int64_t numel, uint32_t* ws_words, float* alpha_out,
@@ -699,50 +425,31 @@ cudaError_t launch_alpha_from_amax(const float* amax, float* alpha, cudaStream_t
 
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float* alpha,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
-    const int64_t prows = padded_rows(rows);
-    const char* tv = getenv("MQ_QUANT_TILES");
-    CUtensorMap xmap;
-    if (!(tv && tv[0] == '0') && make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) {
-        static int sms[64] = {};
-        static bool attr_set[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        const int d = dev < 64 ? dev : 63;
-        if (!attr_set[d]) {
-            cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
-            cudaError_t e = cudaFuncSetAttribute(k_quantize_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
-            if (e != cudaSuccess) return e;
-            e = cudaFuncSetAttribute(k_quantize_ws, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
-            if (e != cudaSuccess) return e;
-            attr_set[d] = true;
-        }
-        const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, 2 * (int64_t)sms[d]));
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        int nattr = 0;
-        set_pdl_attr(attr, &nattr);
-        cfg.gridDim = dim3(grid);
-        cfg.dynamicSmemBytes = QT_SMEM;
-        cfg.stream = stream;
-        cfg.attrs = attr;
-        cfg.numAttrs = nattr;
-        const char* wv = getenv("MQ_QUANT_WS");
-        if (!(wv && wv[0] == '0')) {
-            // the producer/consumer form (MQ_QUANT_WS=0: the block-synchronous ring)
-            cfg.blockDim = dim3(QW_THREADS);
-            return cudaLaunchKernelEx(&cfg, k_quantize_ws, xmap, rows, prows, K, alpha,
-                                      reinterpret_cast<uint4*>(codes), scales);
-        }
-        cfg.blockDim = dim3(QT_THREADS);
-        return cudaLaunchKernelEx(&cfg, k_quantize_tiles, xmap, rows, prows, K, alpha, reinterpret_cast<uint4*>(codes),
-                                  scales);
+    static int sms[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int d = dev < 64 ? dev : 63;
+    if (!sms[d]) {
+        cudaError_t e = cudaFuncSetAttribute(k_quantize_ws, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM);
+        if (e != cudaSuccess) return e;
+        cudaDeviceGetAttribute(&sms[d], cudaDevAttrMultiProcessorCount, dev);
     }
-    const int64_t threads = prows * (K / 64);
-    const int64_t blocks = (threads + QUANT_THREADS - 1) / QUANT_THREADS;
-    k_quantize<<<(unsigned)blocks, QUANT_THREADS, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), rows, prows, K, alpha, reinterpret_cast<uint4*>(codes), scales);
-    return cudaGetLastError();
+    CUtensorMap xmap;
+    if (!make_bf16_tile_map(&xmap, x, rows, K, QT_ROWS)) return cudaErrorInvalidValue;
+    const int64_t prows = padded_rows(rows);
+    const int64_t ntiles = (prows + QT_ROWS - 1) / QT_ROWS * (K / 64);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    int nattr = 0;
+    set_pdl_attr(attr, &nattr);
+    cfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, 2 * (int64_t)sms[d])));
+    cfg.blockDim = dim3(QW_THREADS);
+    cfg.dynamicSmemBytes = QT_SMEM;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = nattr;
+    return cudaLaunchKernelEx(&cfg, k_quantize_ws, xmap, rows, prows, K, alpha, reinterpret_cast<uint4*>(codes),
+                              scales);
 }
 
 }  // namespace mq
