@@ -248,6 +248,25 @@ int mq_linear_w4a4_noalloc(const void *x, int64_t M, int64_t K,
                            void *y, void *stream);
 
 /*
+ * The debug build of the library (libmq_debug.so, the same sources compiled
+ * with MQ_DEBUG=1) checks, before it is made, every global-memory access
+ * that a kernel computes from indices (quantizer code and scale stores, the
+ * fused quantizer's loads and stores, the epilogues' register stores) and
+ * every TMA coordinate and bulk-copy address (the 16-byte rules).  A failed
+ * check counts one hit and skips the access -- nothing traps, the context
+ * stays usable (a skipped copy then shows as MQ_ERR_TIMEOUT on the waits
+ * that expected it).  It stands in for a memory checker on machines where
+ * none may run.
+ *
+ * mq_is_debug_build: 1 in libmq_debug.so, 0 in libmq.so.
+ * mq_debug_bounds_hits: synchronizes the current device, then writes the
+ *   number of failed checks since the previous call into *hits (a host
+ *   pointer) and clears the count; always 0 in the release build.
+ */
+int mq_is_debug_build(void);
+int mq_debug_bounds_hits(int64_t *hits);
+
+/*
  * Synchronizes `stream`, then reads the status word of a workspace into
  * *device_status (MQ_OK or MQ_ERR_TIMEOUT) and clears it.  `ws` is a device
  * pointer, `device_status` a host pointer.

@@ -1,4 +1,5 @@
-"""Build libmq.so (the CUDA kernels and the C ABI) in-tree with nvcc for sm_100a.
+"""Build libmq.so (the CUDA kernels and the C ABI) in-tree with nvcc for sm_100a,
+and libmq_debug.so, the same sources with the bounds checks of MQ_DEBUG.
 
 Usage: python -m nvfp4_w4a4_quantized_03_b200.build [--verbose-ptxas]
 """
@@ -13,6 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmq.so")
+DEBUG_LIB = os.path.join(HERE, "libmq_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -27,22 +29,19 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
     deps.append(os.path.join(HERE, "..", "include", "mq.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    objdir = os.path.join(HERE, "_build")
+def _build_one(lib: str, objdir: str, extra, ptxas_verbose: bool) -> None:
     os.makedirs(objdir, exist_ok=True)
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
-                    "-I", os.path.join(HERE, "..", "include")]
+                    "-I", os.path.join(HERE, "..", "include")] + list(extra)
     if ptxas_verbose:
         flags += ["-Xptxas", "-v"]
     objs = []
@@ -50,9 +49,17 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         subprocess.check_call([nvcc(), "-c", src, "-o", obj] + flags)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     subprocess.check_call([nvcc(), "-shared", "-o", tmp] + objs + ARCH + ["-lcudart_static"])
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Build both libraries if a source is newer (or `force`); returns libmq.so's path."""
+    if force or _stale(LIB):
+        _build_one(LIB, os.path.join(HERE, "_build"), [], ptxas_verbose)
+    if force or _stale(DEBUG_LIB):
+        _build_one(DEBUG_LIB, os.path.join(HERE, "_build", "debug"), ["-DMQ_DEBUG=1"], ptxas_verbose)
     return LIB
 
 

@@ -346,6 +346,24 @@ int mq_debug_gemm_stall(const uint8_t* a_codes, const uint8_t* a_scales, const f
     return cuda_status(mq::launch_gemm(g, sms, static_cast<cudaStream_t>(stream)));
 }
 
+int mq_is_debug_build(void) {
+#ifdef MQ_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int mq_debug_bounds_hits(int64_t* hits) {
+    if (!hits) return MQ_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MQ_ERR_CUDA;
+    const unsigned long long q = mq::debug_hits_quant(), g = mq::gemm::debug_hits_gemm(),
+                             d = mq::decode::debug_hits_decode();
+    if (q == ~0ull || g == ~0ull || d == ~0ull) return MQ_ERR_CUDA;
+    *hits = (int64_t)(q + g + d);
+    return MQ_OK;
+}
+
 int mq_read_status(void* ws, void* stream, int32_t* device_status) {
     if (!ws || !device_status) return MQ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

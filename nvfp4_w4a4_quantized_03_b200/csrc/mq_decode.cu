@@ -27,6 +27,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "mq_debug.cuh"
 #include "mq_internal.h"
 #include "mq_ptx.cuh"
 
@@ -151,11 +152,16 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             for (int kt = kt0; kt < kt1; ++kt) {
                 if (!mbar_wait_bounded(&s->empty[st], phase ^ 1, p.timeout, abort_flag)) { raise(); break; }
                 pending &= ~(1u << st);
-                if (skip) {
-                    skip = false;       // this stage never completes: every wait on it runs out
+                const int nkb = min(NKB, p.kblocks - kt * NKB);
+                const int64_t ka = (int64_t)kt * NKB;
+                if (skip || !MQ_CHECK_TMA_X(kt * 128, 1) || !MQ_CHECK(ka + nkb <= p.katoms && wt < p.w_row_tiles) ||
+                    !MQ_CHECK_BULK(p.w_scales + (wt * p.katoms + ka) * 512, nkb * 512) ||
+                    !MQ_CHECK_BULK(p.x_scales + ka * 512, nkb * 512)) {
+                    // failure-detection test hook (or, in the debug build, a copy
+                    // that would leave the operands): this stage never completes,
+                    // every wait on it runs out
+                    skip = false;
                 } else {
-                    const int nkb = min(NKB, p.kblocks - kt * NKB);
-                    const int64_t ka = (int64_t)kt * NKB;
                     mbar_arrive_expect_tx(&s->ready[st], W_BYTES + p.MP * 128);
                     tma_load_2d(stage_w(st), &tmap_w, &s->ready[st], kt * 128, n0);
                     tma_load_2d(stage_x(st), &tmap_x, &s->ready[st], kt * 128, 0);
@@ -271,7 +277,8 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             for (int m = (int)rank; m < p.M; m += p.split) {
                 float acc = peer[0][m * ROWS + r];
                 for (int q = 1; q < p.split; ++q) acc += peer[q][m * ROWS + r];
-                p.y[(int64_t)m * p.N + n] = __float2bfloat16_rn(__fmul_rn(acc, ab));
+                if (MQ_CHECK((int64_t)m * p.N + n < (int64_t)p.M * p.N))
+                    p.y[(int64_t)m * p.N + n] = __float2bfloat16_rn(__fmul_rn(acc, ab));
             }
         }
     }
@@ -285,6 +292,8 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         tmem_dealloc(tmem, TMEM_COLS);
     }
 }
+
+MQ_DEBUG_READER(debug_hits_decode)
 
 }  // namespace decode
 

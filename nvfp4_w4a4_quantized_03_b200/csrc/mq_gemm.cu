@@ -59,6 +59,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "mq_debug.cuh"
 #include "mq_internal.h"
 #include "mq_nvfp4.cuh"
 #include "mq_ptx.cuh"
@@ -345,7 +346,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         break;
                     }
                     pending &= ~(1u << st);
-                    if (skip) {     // failure-detection test hook: never complete this stage
+                    if (skip || !MQ_CHECK_TMA_X(kt * C::ROW_BYTES, 1) || !MQ_CHECK_TMA_X(kt * NKB * 64, 8)) {
+                        // failure-detection test hook (or, in the debug build, a
+                        // coordinate the TMA would refuse): never complete this stage
                         skip = false;
                     } else {
                         const int64_t ka = (int64_t)kt * NKB;              // first k-atom of the stage
@@ -506,7 +509,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int row = slab * 32 + (batch * 8 + j) * 2 + half;
-                        if (row < p.M && col_ok) {
+                        if (row < p.M && col_ok && MQ_CHECK((int64_t)row * p.K + kb * 16 + 16 <= (int64_t)p.M * p.K)) {
                             const uint4* src = reinterpret_cast<const uint4*>(p.x + (int64_t)row * p.K + kb * 16);
                             v[j][0] = src[0];
                             v[j][1] = src[1];
@@ -521,14 +524,16 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         uint32_t c0 = 0, c1 = 0, sc = 0;
                         if (row < p.M && col_ok) {
                             sc = quantize_block16(v[j][0], v[j][1], alpha, c0, c1);
-                            *reinterpret_cast<uint2*>(p.x_codes + (int64_t)row * (p.K / 2) + kb * 8) =
-                                make_uint2(c0, c1);
+                            if (MQ_CHECK((int64_t)row * (p.K / 2) + kb * 8 + 8 <= (int64_t)p.M * (p.K / 2)))
+                                *reinterpret_cast<uint2*>(p.x_codes + (int64_t)row * (p.K / 2) + kb * 8) =
+                                    make_uint2(c0, c1);
                         }
                         // four consecutive block columns form one 32-bit scale word
                         uint32_t word = sc << (8 * (kbl & 3));
                         word |= __shfl_xor_sync(0xffffffffu, word, 1);
                         word |= __shfl_xor_sync(0xffffffffu, word, 2);
-                        if ((kbl & 3) == 0 && col_ok)
+                        if ((kbl & 3) == 0 && col_ok &&
+                            MQ_CHECK(row < p.a_row_tiles * 128 && kb / 4 < p.katoms))
                             *reinterpret_cast<uint32_t*>(p.x_scales + scale_byte_offset(row, kb, p.katoms)) = word;
                     }
                 }
@@ -656,7 +661,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 fence_proxy_async_shared();
                 __syncwarp();
                 const int hcol = nb * 128 + half * 64;
-                if (lane == 0 && row0 < p.M) {
+                if (lane == 0 && row0 < p.M && MQ_CHECK_TMA_STORE(hcol, row0, 2)) {
                     tma_store_2d(&tmap_y, box, hcol, row0);
                     bulk_commit_group();
                 }
@@ -680,7 +685,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 auto issue = [&](int h) {
                     fence_proxy_async_shared();
                     __syncwarp();
-                    if (lane == 0 && row0 < p.M && colh + h * 64 < p.N) {
+                    if (lane == 0 && row0 < p.M && colh + h * 64 < p.N && MQ_CHECK_TMA_STORE(colh + h * 64, row0, 2)) {
                         tma_store_2d(&tmap_y, box, colh + h * 64, row0);
                         bulk_commit_group();
                     }
@@ -739,7 +744,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
-                if (row < p.M) {
+                if (row < p.M && MQ_CHECK((int64_t)row * p.N + colh + 128 <= (int64_t)p.M * p.N)) {
                     uint4* d4 = reinterpret_cast<uint4*>(p.y + (int64_t)row * p.N + colh);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
@@ -765,7 +770,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     uint16_t* d16 = reinterpret_cast<uint16_t*>(p.y + (int64_t)row * p.N + col0);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        if (col0 + j < p.N) {
+                        if (col0 + j < p.N && MQ_CHECK((int64_t)row * p.N + col0 + j < (int64_t)p.M * p.N)) {
                             const uint32_t two = cvt_bf16x2(0.0f, __fmul_rn(__uint_as_float(r[j]), ab));
                             d16[j] = (uint16_t)(two & 0xffffu);
                         }
@@ -787,6 +792,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         else tmem_dealloc(tmem, TMEM_COLS);
     }
 }
+
+MQ_DEBUG_READER(debug_hits_gemm)
 
 }  // namespace gemm
 

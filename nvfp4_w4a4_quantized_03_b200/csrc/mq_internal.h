@@ -82,6 +82,12 @@ struct GemmArgs {
     uint32_t* h_amax = nullptr;
 };
 
+// Debug build (MQ_DEBUG): bounds-check hits of each translation unit since
+// its last read (0 in the release build).
+unsigned long long debug_hits_quant();
+namespace gemm { unsigned long long debug_hits_gemm(); }
+namespace decode { unsigned long long debug_hits_decode(); }
+
 // Readiness flags of the fused linear: one int per (128-row block, K stage).
 int64_t fused_flag_count(int64_t M, int64_t K);
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);

@@ -24,6 +24,7 @@
 #include <algorithm>
 #include <cstdlib>
 
+#include "mq_debug.cuh"
 #include "mq_internal.h"
 #include "mq_nvfp4.cuh"
 
@@ -131,7 +132,8 @@ __device__ __forceinline__ void quantize_quad(int64_t rows, int64_t K, uint32_t 
 #pragma unroll
         for (int b = 0; b < 4; ++b) word |= quantize_block16(v[2 * b], v[2 * b + 1], alpha, c[2 * b], c[2 * b + 1]) << (8 * b);
         uint4* dst = codes + ((int64_t)row * (K / 64) + q) * 2;      // 32 bytes per quad
-        if ((reinterpret_cast<uintptr_t>(codes) & 31) == 0) {
+        if (!MQ_CHECK(q < (uint32_t)(K / 64))) {
+        } else if ((reinterpret_cast<uintptr_t>(codes) & 31) == 0) {
             asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(c[0]), "r"(c[1]),
                          "r"(c[2]), "r"(c[3]), "r"(c[4]), "r"(c[5]), "r"(c[6]), "r"(c[7]) : "memory");
         } else {
@@ -139,7 +141,8 @@ __device__ __forceinline__ void quantize_quad(int64_t rows, int64_t K, uint32_t 
             dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
         }
     }
-    *reinterpret_cast<uint32_t*>(scales + scale_byte_offset(row, 4 * (int64_t)q, K / 64)) = word;
+    if (MQ_CHECK(row < padded_rows(rows) && q < (uint32_t)(K / 64)))
+        *reinterpret_cast<uint32_t*>(scales + scale_byte_offset(row, 4 * (int64_t)q, K / 64)) = word;
 }
 
 // ---------------------------------------------------------------------------
@@ -201,8 +204,9 @@ k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t pr
                 if (round > 0 && !mbar_wait_bounded(&empty[st], (round - 1) & 1, timeout, nullptr)) break;
                 const int64_t t = blockIdx.x + i * gridDim.x;
                 mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
-                tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
-                            (int32_t)(t / kgroups) * QT_ROWS);
+                if (MQ_CHECK_TMA_X((t % kgroups) * 64, 2))
+                    tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
+                                (int32_t)(t / kgroups) * QT_ROWS);
             }
             // every copy this thread issued lands before the block ends
             for (int64_t j = i > QT_STAGES ? i - QT_STAGES : 0; j < i; ++j)
@@ -278,8 +282,9 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
                 if (round > 0 && !mbar_wait_bounded(&empty[st], (round - 1) & 1, timeout, nullptr)) break;
                 const int64_t t = box_of(item);
                 mbar_arrive_expect_tx(&full[st], QT_BOX_BYTES);
-                tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
-                            (int32_t)(t / kgroups) * QT_ROWS);
+                if (MQ_CHECK_TMA_X((t % kgroups) * 64, 2))
+                    tma_load_2d(base + st * QT_BOX_BYTES, &xmap, &full[st], (int32_t)(t % kgroups) * 64,
+                                (int32_t)(t / kgroups) * QT_ROWS);
             }
             // every copy this thread issued lands before the block ends
             for (int64_t j = item > QT_STAGES ? item - QT_STAGES : 0; j < item; ++j)
@@ -451,5 +456,7 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, const float*
     return cudaLaunchKernelEx(&cfg, k_quantize_ws, xmap, rows, prows, K, alpha, reinterpret_cast<uint4*>(codes),
                               scales);
 }
+
+MQ_DEBUG_READER(debug_hits_quant)
 
 }  // namespace mq

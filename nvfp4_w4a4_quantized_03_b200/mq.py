@@ -6,6 +6,8 @@ not been built or the current device is not a B200 (sm_100a), calls raise.
 
 The functions keep the C names.  They take torch CUDA tensors (for device
 memory) and enqueue on the current torch stream unless `stream` is given.
+With MQ_DEBUG=1 in the environment the debug build (libmq_debug.so, every
+index-computed access and TMA coordinate bounds-checked) is loaded instead.
 """
 from __future__ import annotations
 
@@ -15,7 +17,7 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmq.so")
+LIB_PATH = os.path.join(_HERE, "libmq_debug.so" if os.environ.get("MQ_DEBUG") == "1" else "libmq.so")
 
 MQ_OK = 0
 MQ_ERR_TIMEOUT = -7
@@ -56,9 +58,11 @@ def lib() -> ctypes.CDLL:
         L.mq_mlp_w4a4_workspace_bytes.argtypes = [i64, i64, i64]
         L.mq_mlp_w4a4_workspace_bytes.restype = sz
         L.mq_mlp_w4a4.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, sz, vp]
+        L.mq_is_debug_build.argtypes = []
+        L.mq_debug_bounds_hits.argtypes = [ctypes.POINTER(ctypes.c_int64)]
         for name in ("mq_tensor_scale", "mq_tensor_amax", "mq_alpha_from_amax", "mq_nvfp4_quantize",
                      "mq_nvfp4_gemm", "mq_linear_w4a4", "mq_read_status", "mq_nvfp4_gemm_swiglu",
-                     "mq_mlp_w4a4"):
+                     "mq_mlp_w4a4", "mq_is_debug_build", "mq_debug_bounds_hits"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -169,6 +173,18 @@ def mq_mlp_w4a4(x: torch.Tensor, wgu_codes, wgu_scales, alpha_gu, inter: int, wd
     _check(lib().mq_mlp_w4a4(_ptr(x), M, K, _ptr(wgu_codes), _ptr(wgu_scales), _ptr(alpha_gu), inter,
                              _ptr(wd_codes), _ptr(wd_scales), _ptr(alpha_d), N, _ptr(y), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "mq_mlp_w4a4")
+
+
+def mq_is_debug_build() -> bool:
+    return bool(lib().mq_is_debug_build())
+
+
+def mq_debug_bounds_hits() -> int:
+    """Failed bounds checks since the previous call (synchronizes the device;
+    always 0 in the release build)."""
+    out = ctypes.c_int64(0)
+    _check(lib().mq_debug_bounds_hits(ctypes.byref(out)), "mq_debug_bounds_hits")
+    return int(out.value)
 
 
 def mq_read_status(ws: torch.Tensor, stream=None) -> int:

@@ -107,3 +107,16 @@ def test_noalloc_constant_and_host_checks(libmq):
     assert f(None, 128, 1024, p16, p16, p16, 256, p16, None) == -1               # null
     assert f(vp(4097), 128, 1024, p16, p16, p16, 256, p16, None) == -3           # misaligned
     assert f(p16, 131072, 4096, p16, p16, p16, 256, p16, None) == -5             # beyond the scratch
+
+
+def test_debug_build_exports_the_same_symbols(libmq):
+    """libmq_debug.so (the MQ_DEBUG bounds-check build) exports every
+    declared entry point and reports itself as the debug build."""
+    from nvfp4_w4a4_quantized_03_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.DEBUG_LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(mq_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, missing
+    dbg = ctypes.CDLL(build.DEBUG_LIB)
+    assert dbg.mq_is_debug_build() == 1
+    assert libmq.mq_is_debug_build() == 0
