@@ -23,9 +23,10 @@
 //               of the scale array viewed as 64-bit words (A's slice, and B's
 //               two slices in one 2-row box), completing on this CTA's
 //               sf_full: four copies per stage.
-//   warp 1      allocates TMEM; in the (even) CTA one lane issues
-//               tcgen05.mma (K = 64 per instruction, 4 per stage) and
-//               tcgen05.commit to release stages and to publish a tile.
+//   warp 1      allocates TMEM; in the (even) CTA the whole warp runs the
+//               MMA loop and an elected lane issues tcgen05.mma (K = 64 per
+//               instruction, 4 per stage, back to back) and tcgen05.commit
+//               to release stages and to publish a tile.
 //   warps 2..3  fused linear only (QUANT): quantizer warps.  They quantize the
 //               bf16 activation X into A's codes and scales (mq_nvfp4.cuh),
 //               32 rows x one K stage at a time, in the order the tile raster
@@ -416,12 +417,18 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && rank == 0) {
+        // The whole warp runs the loop, so its state (stage, phase, the
+        // operands) is warp-uniform; one elected lane issues the MMAs and the
+        // commits.  With a single lane running it alone, the per-stage issue
+        // took ~360 SM cycles instead of ~200 (clock64 traces): the
+        // operands had to be moved into place before every MMA.
+        const bool leader = elect_one();
+        if (rank == 0) {
             int st = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int tile = unit; tile < p.tiles && !*abort_flag; tile += units) {
-                if (!mbar_wait_bounded(&s->acc_empty, acc_phase ^ 1, p.timeout, abort_flag)) {
-                    raise_abort(s, p);
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s->acc_empty, acc_phase ^ 1, p.timeout, abort_flag))) {
+                    if (leader) raise_abort(s, p);
                     break;
                 }
                 tc_fence_after();
@@ -429,50 +436,77 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 // its scales in TMEM), then its MMAs back to back, then the
                 // commit that frees the stage.  Any other instruction between
                 // two MMAs -- even a branch not taken, let alone a barrier
-                // poll -- costs the tensor pipe ~30-60 cycles per MMA (clock64
-                // traces: 773 SM cycles per 4-MMA stage with the next stage's
-                // wait placed before the last MMA, 700 with this order, 512
-                // back to back), so the waits sit only at stage boundaries.
+                // poll or operand arithmetic -- costs the tensor pipe 30-60
+                // cycles per MMA (clock64 traces: 773 SM cycles per 4-MMA
+                // stage with the next stage's wait placed before the last MMA,
+                // 700 with the wait at the boundary, 656 with the operands
+                // computed ahead, ~590 issued by the whole warp, where the
+                // per-SM load intake becomes the limit), so the waits sit only
+                // at stage boundaries and the next stage's operands are
+                // computed while the current stage's MMAs run.
                 bool ok = true;
-                for (int kt = 0; kt < p.k_stages; ++kt) {
-                    if (!mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const int nkb = min(NKB, p.kblocks - kt * NKB);
-                    const uint64_t ad0 = smem_desc(smem_u32(stage_a(st)), 16, C::SBO, C::SWIZZLE);
-                    const uint64_t bd0 = smem_desc(smem_u32(stage_b(st)), 16, C::SBO, C::SWIZZLE);
-                    const uint32_t sf = tmem + SF_COL + st * SF_COLS_PER_STAGE;
-                    const uint32_t acc0 = kt != 0;
-                    auto mma = [&](int kb, uint32_t acc) {
-                        const uint64_t step = (uint64_t)(kb * (MMA_K / 2) >> 4);
-                        if (PAIR == 2)
-                            mma_mxf4nvf4_pair(tmem + ACC_COL, ad0 + step, bd0 + step, C::IDESC, sf + kb * 4,
-                                              sf + SFB_OFF + kb * 8, acc);
-                        else
-                            mma_mxf4nvf4(tmem + ACC_COL, ad0 + step, bd0 + step, C::IDESC, sf + kb * 4,
-                                         sf + SFB_OFF + kb * 8, acc);
-                    };
-                    if (nkb == NKB) {
-                        // a full stage: straight-line code from the first MMA to the last
-                        mma(0, acc0);
+                // operands of a stage: both descriptors and both scale addresses of each MMA
+                uint64_t opa[NKB], opb[NKB];
+                uint32_t osa[NKB], osb[NKB];
+                auto prep = [&](int stg) {
+                    const uint64_t ad0 = smem_desc(smem_u32(stage_a(stg)), 16, C::SBO, C::SWIZZLE);
+                    const uint64_t bd0 = smem_desc(smem_u32(stage_b(stg)), 16, C::SBO, C::SWIZZLE);
+                    const uint32_t sf = tmem + SF_COL + stg * SF_COLS_PER_STAGE;
 #pragma unroll
-                        for (int kb = 1; kb < NKB; ++kb) mma(kb, 1u);
-                    } else {
-                        for (int kb = 0; kb < nkb; ++kb) mma(kb, (kt | kb) != 0);
+                    for (int kb = 0; kb < NKB; ++kb) {
+                        opa[kb] = ad0 + (uint64_t)(kb * (MMA_K / 2) >> 4);
+                        opb[kb] = bd0 + (uint64_t)(kb * (MMA_K / 2) >> 4);
+                        osa[kb] = sf + kb * 4;
+                        osb[kb] = sf + SFB_OFF + kb * 8;
                     }
-                    commit_to_all<PAIR>(&s->empty[st]);
+                };
+                auto mma = [&](int kb, uint32_t acc) {
+                    if (PAIR == 2)
+                        mma_mxf4nvf4_pair(tmem + ACC_COL, opa[kb], opb[kb], C::IDESC, osa[kb], osb[kb], acc);
+                    else
+                        mma_mxf4nvf4(tmem + ACC_COL, opa[kb], opb[kb], C::IDESC, osa[kb], osb[kb], acc);
+                };
+                prep(st);
+                const int full_stages = p.kblocks / NKB;        // stages with all NKB MMAs
+                for (int kt = 0; kt < p.k_stages; ++kt) {
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (leader) {
+                        if (kt < full_stages) {
+                            mma(0, kt != 0);
+                            mma(1, 1u);
+                            mma(2, 1u);
+                            mma(3, 1u);
+                        } else {
+                            const int nkb = p.kblocks - kt * NKB;
+#pragma unroll
+                            for (int kb = 0; kb < NKB; ++kb)
+                                if (kb < nkb) mma(kb, (kt | kb) != 0);
+                        }
+                        commit_to_all<PAIR>(&s->empty[st]);
+                    }
+                    __syncwarp();
                     st = st + 1 == p.stages ? 0 : st + 1;
                     phase = st == 0 ? phase ^ 1 : phase;
+                    prep(st);
                 }
                 if (!ok) {
-                    raise_abort(s, p);
+                    if (leader) raise_abort(s, p);
                     break;
                 }
-                commit_to_all<PAIR>(&s->acc_full);
+                if (leader) commit_to_all<PAIR>(&s->acc_full);
+                __syncwarp();
                 acc_phase ^= 1;
             }
             // no MMA may still be running when TMEM is released
-            if (PAIR == 2) mma_commit_pair_mc(&s->drain, 0x1);
-            else mma_commit(&s->drain);
+            if (leader) {
+                if (PAIR == 2) mma_commit_pair_mc(&s->drain, 0x1);
+                else mma_commit(&s->drain);
+            }
+            __syncwarp();
             mbar_wait_bounded(&s->drain, 0, p.timeout, nullptr);
         }
     } else if (warp < FIRST_SF_WARP) {
