@@ -74,6 +74,50 @@ __device__ __forceinline__ uint32_t quantize_block16(const uint4& v0, const uint
     return sc;
 }
 
+// The per-tensor constants of the table-driven form below, set once alpha
+// is known: d = fl32(6 alpha), and rtab[c] = RN(1 / fl32(alpha sigma(c)))
+// for every E4M3 code c (entry 0 unused) -- the same operations
+// quantize_block16 performs per block, so both forms give the same bits.
+struct QuantTab {
+    float d;
+    const float* rtab;
+};
+
+// Fills rtab (128 floats, shared memory) with thread `i` of `n` threads.
+__device__ __forceinline__ void fill_recip_table(float* rtab, float alpha, int i, int n) {
+    for (int c = i; c < 128; c += n) {
+        const float sigma = __half2float(__ushort_as_half((uint16_t)(cvt_e4m3x2_to_f16x2((uint16_t)c) & 0xffffu)));
+        rtab[c] = c == 0 ? 0.0f : __frcp_rn(__fmul_rn(alpha, sigma));
+    }
+}
+
+// quantize_block16 with the same results, fewer instructions: the
+// reciprocal of fl32(alpha sigma_b) read from the table instead of computed
+// per block, and d = fl32(6 alpha) computed once.
+__device__ __forceinline__ uint32_t quantize_block16_tab(const uint4& v0, const uint4& v1, const QuantTab& qt,
+                                                         uint32_t& c0, uint32_t& c1) {
+    uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v0.x, v0.y), absmax_bf16x2(v0.z, v0.w)),
+                               absmax_bf16x2(absmax_bf16x2(v1.x, v1.y), absmax_bf16x2(v1.z, v1.w)));
+    m &= 0x7fff7fffu;
+    const float amax_b = __uint_as_float(max(m & 0xffffu, m >> 16) << 16);
+    const float t = __fdiv_rn(amax_b, qt.d);
+    const uint32_t sc = cvt_e4m3x2(0.0f, t) & 0xffu;
+    c0 = 0;
+    c1 = 0;
+    if (sc != 0) {
+        const float r = qt.rtab[sc];
+        uint64_t rr;
+        asm("mov.b64 %0, {%1, %1};" : "=l"(rr) : "f"(r));
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) scale_bf16x2(w[i], rr, f[2 * i], f[2 * i + 1]);
+        c0 = cvt_e2m1x8(f[0], f[1], f[2], f[3], f[4], f[5], f[6], f[7]);
+        c1 = cvt_e2m1x8(f[8], f[9], f[10], f[11], f[12], f[13], f[14], f[15]);
+    }
+    return sc;
+}
+
 // Byte offset of (row, scale column kb) in the MMA scale layout: atoms of
 // 128 rows x 4 columns, ordered row-tile major; inside an atom row r sits at
 // (r % 32) * 16 + ((r / 32) % 4) * 4 and column kb at kb % 4.

@@ -123,14 +123,14 @@ k_amax(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ t
 // sector per request instead of two half-sector writes, which took the
 // stand-alone quantizer on 8192 x 12288 from 51 to 45 us (the threads of a
 // warp write 32 different rows, so no two stores of a warp share a sector).
-__device__ __forceinline__ void quantize_quad(int64_t rows, int64_t K, uint32_t row, uint32_t q, float alpha,
+__device__ __forceinline__ void quantize_quad(int64_t rows, int64_t K, uint32_t row, uint32_t q, const QuantTab& qt,
                                               uint4* __restrict__ codes, uint8_t* __restrict__ scales,
                                               const uint4 (&v)[8]) {
     uint32_t word = 0;
     if (row < rows) {
         uint32_t c[8];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) word |= quantize_block16(v[2 * b], v[2 * b + 1], alpha, c[2 * b], c[2 * b + 1]) << (8 * b);
+        for (int b = 0; b < 4; ++b) word |= quantize_block16_tab(v[2 * b], v[2 * b + 1], qt, c[2 * b], c[2 * b + 1]) << (8 * b);
         uint4* dst = codes + ((int64_t)row * (K / 64) + q) * 2;      // 32 bytes per quad
         if (!MQ_CHECK(q < (uint32_t)(K / 64))) {
         } else if ((reinterpret_cast<uintptr_t>(codes) & 31) == 0) {
@@ -214,7 +214,13 @@ k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t pr
         }
         return;
     }
+    __shared__ float rtab[QW_CONSUMERS][128];       // one table per quantizing warp
     const float alpha = __ldg(alpha_p);
+    fill_recip_table(rtab[warp], alpha, lane, 32);
+    __syncwarp();
+    QuantTab qt;
+    qt.d = __fmul_rn(6.0f, alpha);
+    qt.rtab = rtab[warp];
     for (int64_t i = 0; i < n; ++i) {
         const int st = (int)(i % QT_STAGES);
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[st], (uint32_t)(i / QT_STAGES) & 1, timeout, nullptr)))
@@ -228,7 +234,7 @@ k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t pr
         if (lane == 0) mbar_arrive(&empty[st]);       // this warp is done with the slot
         const int64_t t = blockIdx.x + i * gridDim.x;
         const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
-        if (row < prows) quantize_quad(rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
+        if (row < prows) quantize_quad(rows, K, (uint32_t)row, (uint32_t)(t % kgroups), qt, codes, scales, v);
     }
 }
 
@@ -297,6 +303,8 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
     uint32_t m = 0;
     float alpha = 0.0f;
     bool ok = true;
+    __shared__ float rtab[QW_CONSUMERS][128];       // one table per quantizing warp
+    QuantTab qt;
     auto boundary = [&]() {
         const uint32_t v = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
         if (lane == 0) {
@@ -317,6 +325,10 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
         }
         const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&alpha_ready, 0, timeout, nullptr));
         alpha = alpha_shared;
+        fill_recip_table(rtab[warp], alpha, lane, 32);
+        __syncwarp();
+        qt.d = __fmul_rn(6.0f, alpha);
+            qt.rtab = rtab[warp];
         ok = got && ok_shared != 0;
     };
     if (n == 0) boundary();
@@ -343,7 +355,7 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
         } else {
             const int64_t t = box_of(item);
             const int64_t row = (t / kgroups) * QT_ROWS + threadIdx.x;
-            if (row < prows) quantize_quad(rows, K, (uint32_t)row, (uint32_t)(t % kgroups), alpha, codes, scales, v);
+            if (row < prows) quantize_quad(rows, K, (uint32_t)row, (uint32_t)(t % kgroups), qt, codes, scales, v);
         }
     }
 }
