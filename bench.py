@@ -806,13 +806,24 @@ def _e2e(args, work, device, stream):
 
 
 def profile_target(which: str):
-    """One gate/up-shaped NVFP4 GEMM (8192 x 24576 x 4096) inside an NVTX
-    range "gemm", after 3 unmarked launches, for `ncu --nvtx --nvtx-include
-    gemm/`: `ours` is mq_nvfp4_gemm on quantized operands, `library` the
-    library NVFP4 GEMM (cuBLASLt through torch._scaled_mm; context for the
-    profile comparison only, on random codes and unit scales)."""
+    """One gate/up-shaped (8192 x 24576 x 4096) launch inside an NVTX range
+    "gemm", after 3 unmarked ones, for `ncu --nvtx --nvtx-include gemm/`:
+    `ours` is mq_nvfp4_gemm on quantized operands, `linear` the linear
+    mq_linear_w4a4 (k_quantize_onepass_ws + k_gemm), `ingemm` the linear with
+    the activation quantized by the GEMM's own quantizer warps (k_amax +
+    k_gemm with quantizer warps), `library` the library NVFP4 GEMM (cuBLASLt
+    through torch._scaled_mm; context for the profile comparison only, on
+    random codes and unit scales)."""
     M, N, K = TOKENS, 24576, 4096
-    if which == "library":
+    if which in ("linear", "ingemm"):
+        from nvfp4_w4a4_quantized_03_b200 import mq
+        if which == "ingemm":
+            os.environ["MQ_LINEAR_PATH"] = "ingemm"
+        x = inputs.activation_bf16(M, K, seed=1, outlier_channels=inputs.outlier_count(K), device="cuda")
+        lin = mq.LinearW4A4(inputs.weight_bf16(N, K, seed=2, device="cuda"))
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        f = lambda: lin(x, y)
+    elif which == "library":
         a = torch.randint(0, 255, (M, K // 2), dtype=torch.uint8, device="cuda").view(torch.float4_e2m1fn_x2)
         b = torch.randint(0, 255, (N, K // 2), dtype=torch.uint8, device="cuda").view(torch.float4_e2m1fn_x2)
         sa = torch.full((M * K // 16,), 1.0, device="cuda").to(torch.float8_e4m3fn)
@@ -844,8 +855,8 @@ def main():
     ap.add_argument("--no-sequence", action="store_true",
                     help="skip the figures beside the metric (36-layer x 131072-token prefill sequence, decode, "
                          "MLP, small linear, 32768-token projections, shape sweep)")
-    ap.add_argument("--profile-target", choices=["ours", "library"], default=None,
-                    help="run one gate/up GEMM in an NVTX range for ncu and exit (no timing)")
+    ap.add_argument("--profile-target", choices=["ours", "linear", "ingemm", "library"], default=None,
+                    help="run one gate/up-shaped GEMM or linear in an NVTX range for ncu and exit (no timing)")
     args = ap.parse_args()
     if args.profile_target:
         profile_target(args.profile_target)
