@@ -76,12 +76,14 @@ def _peaks():
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running (every
     half millisecond, so that even a timed region of ~15 ms gets 20 or more
-    samples)."""
+    samples).  Entering waits until NVML is up and the first sample is taken,
+    so the samples cover the region that follows."""
 
     def __init__(self, index: int, period_s: float = 0.0005):
         self.index, self.period = index, period_s
         self.samples, self.reasons = [], set()
         self._stop = threading.Event()
+        self._ready = threading.Event()
         self._t = None
         self.max_mhz = None
 
@@ -99,13 +101,18 @@ class ClockSampler:
                 for name, bit in flags.items():
                     if r & bit:
                         self.reasons.add(name)
+                self._ready.set()
                 time.sleep(self.period)
         except Exception as e:  # pragma: no cover - NVML missing
             self.reasons.add(f"nvml-unavailable: {type(e).__name__}")
+        finally:
+            self._ready.set()
 
     def __enter__(self):
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
+        self._ready.wait(timeout=10.0)
+        del self.samples[:len(self.samples)]     # taken before the region
         return self
 
     def __exit__(self, *a):
