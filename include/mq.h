@@ -290,6 +290,66 @@ int mq_debug_gemm_stall(const uint8_t *a_codes, const uint8_t *a_scales, const f
                         int64_t M, int64_t N, int64_t K, void *y, void *ws, size_t ws_bytes,
                         int64_t timeout_cycles, void *stream);
 
+/*
+ * Test hook for the allocation-free entry point; the paper has no
+ * counterpart.  Enqueues on `stream` a fill of the header words of the
+ * current device's static scratch (its grid-barrier ticket, running max,
+ * generation and status words) with the 32-bit `word`, the state that a
+ * call ended by MQ_ERR_TIMEOUT can leave behind.  The next
+ * mq_linear_w4a4_noalloc call clears the header before its kernels run, so
+ * its result does not depend on what this wrote.  Returns MQ_OK or
+ * MQ_ERR_CUDA.
+ */
+int mq_debug_noalloc_fill_header(uint32_t word, void *stream);
+
+/*
+ * Selectable alternatives.  Each switch picks among kernels or launch
+ * shapes that compute the same result (the tests compare their outputs bit
+ * for bit); the defaults are the fastest measured.  A switch is one
+ * process-wide value: mq_set_switch takes effect for launches enqueued after
+ * it returns, from any thread.  The first call into the library sets every
+ * switch from its environment variable (named beside it), once; later
+ * changes of the environment have no effect.
+ *
+ *   MQ_SWITCH_LINEAR_PATH   (MQ_LINEAR_PATH: onepass | split | ingemm)
+ *       how mq_linear_w4a4 quantizes X: 0 one cooperative kernel (amax, grid
+ *       barrier, quantization; default), 1 the mq_tensor_scale and
+ *       mq_nvfp4_quantize kernels, 2 the amax kernel and quantizer warps
+ *       inside the GEMM.
+ *   MQ_SWITCH_GEMM_FORM     (MQ_GEMM_FORM: 1 | 2)
+ *       0 by rule (CTA pairs for M > 128, else one CTA; the decode form for
+ *       M <= 64), 1 the one-CTA prefill form, 2 the CTA-pair form.
+ *   MQ_SWITCH_GEMM_DECODE   (MQ_GEMM_DECODE: 0 | 1)
+ *       1 the split-K decode form for M <= 64 (default), 0 the prefill form.
+ *   MQ_SWITCH_DECODE_SPLIT  (MQ_DECODE_SPLIT: 1 | 2 | 4 | 8)
+ *       0 split-K of the decode form by rule, else that split (at most the
+ *       number of 256-K stages).
+ *   MQ_SWITCH_GEMM_STAGES   (MQ_GEMM_STAGES)
+ *       0 every pipeline stage the prefill form has room for, else 2.. that
+ *       many (fewer than the room are used as is).
+ *   MQ_SWITCH_GEMM_GROUP_M  (MQ_GEMM_GROUP_M)
+ *       0 the default tile raster (32 M-blocks per group), else 1 .. 2^20.
+ *   MQ_SWITCH_PDL           (MQ_PDL: 0 | 1)
+ *       1 launches carry programmatic dependent launch (default), 0 not.
+ *
+ * mq_set_switch returns MQ_OK, or MQ_ERR_INVALID_ARG for an unknown switch
+ * or a value outside its range (the switch keeps its value).
+ * mq_get_switch returns the value, or MQ_ERR_INVALID_ARG for an unknown
+ * switch.
+ */
+enum {
+    MQ_SWITCH_LINEAR_PATH = 0,
+    MQ_SWITCH_GEMM_FORM = 1,
+    MQ_SWITCH_GEMM_DECODE = 2,
+    MQ_SWITCH_DECODE_SPLIT = 3,
+    MQ_SWITCH_GEMM_STAGES = 4,
+    MQ_SWITCH_GEMM_GROUP_M = 5,
+    MQ_SWITCH_PDL = 6,
+    MQ_SWITCH_COUNT = 7
+};
+int mq_set_switch(int which, int value);
+int mq_get_switch(int which);
+
 #ifdef __cplusplus
 }
 #endif

@@ -3,6 +3,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/mq.h"
@@ -64,14 +65,58 @@ int check_linear_shape(int64_t M, int64_t N, int64_t K) {
     return st != MQ_OK ? st : check_rows_k(N, K);
 }
 
-bool pdl_enabled() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = getenv("MQ_PDL");
-        v = (e && e[0] == '0') ? 0 : 1;
-    }
-    return v == 1;
+namespace {
+
+// Range of each switch (include/mq.h) and its environment variable.
+struct SwitchDef {
+    const char* env;
+    int lo, hi, dflt;
+};
+constexpr SwitchDef SWITCH_DEFS[MQ_SWITCH_COUNT] = {
+    {"MQ_LINEAR_PATH", 0, 2, 0},        // onepass | split | ingemm
+    {"MQ_GEMM_FORM", 0, 2, 0},          // rule | one CTA | CTA pair
+    {"MQ_GEMM_DECODE", 0, 1, 1},
+    {"MQ_DECODE_SPLIT", 0, 8, 0},       // rule | 1, 2, 4, 8
+    {"MQ_GEMM_STAGES", 0, 64, 0},       // every stage | 2 ..
+    {"MQ_GEMM_GROUP_M", 0, 1 << 20, 0}, // default raster | 1 ..
+    {"MQ_PDL", 0, 1, 1},
+};
+
+bool switch_value_ok(int which, int v) {
+    const SwitchDef& d = SWITCH_DEFS[which];
+    if (v < d.lo || v > d.hi) return false;
+    if (which == MQ_SWITCH_DECODE_SPLIT) return v == 0 || v == 1 || v == 2 || v == 4 || v == 8;
+    if (which == MQ_SWITCH_GEMM_STAGES) return v == 0 || v >= 2;
+    return true;
 }
+
+// The environment's value of a switch (its default when unset or invalid).
+int switch_from_env(int which) {
+    const SwitchDef& d = SWITCH_DEFS[which];
+    const char* e = getenv(d.env);
+    if (!e || !e[0]) return d.dflt;
+    if (which == MQ_SWITCH_LINEAR_PATH) return e[0] == 's' ? 1 : e[0] == 'i' ? 2 : 0;
+    const int v = atoi(e);
+    return switch_value_ok(which, v) ? v : d.dflt;
+}
+
+std::atomic<int> g_switch[MQ_SWITCH_COUNT];
+std::once_flag g_switch_once;
+
+void init_switches() {
+    std::call_once(g_switch_once, [] {
+        for (int i = 0; i < MQ_SWITCH_COUNT; ++i) g_switch[i].store(switch_from_env(i), std::memory_order_relaxed);
+    });
+}
+
+}  // namespace
+
+int switch_value(int which) {
+    init_switches();
+    return g_switch[which].load(std::memory_order_relaxed);
+}
+
+bool pdl_enabled() { return switch_value(MQ_SWITCH_PDL) == 1; }
 void set_pdl_attr(cudaLaunchAttribute* attr, int* nattr) {
     if (!pdl_enabled()) return;
     attr[*nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -215,21 +260,20 @@ int mq_linear_w4a4(const void* x, int64_t M, int64_t K, const uint8_t* w_codes, 
     uint8_t* x_scales = x_codes + round256(mq_nvfp4_codes_bytes(M, K));
     mq::GemmArgs g{x_codes, x_scales, alpha_x, w_codes, w_scales, alpha_w, y, M, N, K,
                    reinterpret_cast<int*>(words + mq::WS_STATUS), DEFAULT_TIMEOUT_CYCLES, 0};
-    // MQ_LINEAR_PATH selects how X is quantized (all three give identical Y):
-    //   "onepass" (default) one cooperative kernel: amax, grid barrier,
-    //                       quantization of the data the amax pass left in L2;
-    //   "split"             mq_tensor_scale's and mq_nvfp4_quantize's kernels;
-    //   "ingemm"            amax kernel, then quantizer warps inside the GEMM.
-    const char* path = getenv("MQ_LINEAR_PATH");
-    const char mode = path ? path[0] : 'o';
+    // MQ_SWITCH_LINEAR_PATH selects how X is quantized (all three give identical Y):
+    //   0 (default) one cooperative kernel: amax, grid barrier, quantization
+    //               of the data the amax pass left in L2;
+    //   1           mq_tensor_scale's and mq_nvfp4_quantize's kernels;
+    //   2           amax kernel, then quantizer warps inside the GEMM.
+    const int mode = mq::switch_value(MQ_SWITCH_LINEAR_PATH);
     cudaError_t e = cudaSuccess;
-    if (mode == 'i') {
+    if (mode == 2) {
         // amax (which also clears the readiness flags), then the GEMM with
         // the activation's quantization done by its quantizer warps
         e = mq::launch_amax(x, M * K, words, alpha_x, sms, s, flags, (int)mq::fused_flag_count(M, K));
         g.x = x;
         g.flags = flags;
-    } else if (mode == 's') {
+    } else if (mode == 1) {
         e = mq::launch_amax(x, M * K, words, alpha_x, sms, s);
         if (e == cudaSuccess) e = mq::launch_quantize(x, M, K, alpha_x, x_codes, x_scales, s);
     } else {
@@ -352,6 +396,18 @@ int mq_is_debug_build(void) {
 #else
     return 0;
 #endif
+}
+
+int mq_set_switch(int which, int value) {
+    if (which < 0 || which >= MQ_SWITCH_COUNT || !mq::switch_value_ok(which, value)) return MQ_ERR_INVALID_ARG;
+    mq::init_switches();
+    mq::g_switch[which].store(value, std::memory_order_relaxed);
+    return MQ_OK;
+}
+
+int mq_get_switch(int which) {
+    if (which < 0 || which >= MQ_SWITCH_COUNT) return MQ_ERR_INVALID_ARG;
+    return mq::switch_value(which);
 }
 
 int mq_debug_bounds_hits(int64_t* hits) {

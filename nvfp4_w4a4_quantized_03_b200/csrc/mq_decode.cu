@@ -27,6 +27,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "../../include/mq.h"
 #include "mq_debug.cuh"
 #include "mq_internal.h"
 #include "mq_ptx.cuh"
@@ -339,11 +340,8 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, int num_sms, cudaStream_t stre
     // projection)
     int split = 1;
     while (split < 8 && (int64_t)tiles * split * 2 <= 2 * (int64_t)num_sms && p.k_stages >= 4 * split * 2) split *= 2;
-    const char* sv = getenv("MQ_DECODE_SPLIT");
-    if (sv) {
-        const int f = atoi(sv);
-        if ((f == 1 || f == 2 || f == 4 || f == 8) && f <= p.k_stages) split = f;
-    }
+    const int forced = switch_value(MQ_SWITCH_DECODE_SPLIT);
+    if (forced > 0 && forced <= p.k_stages) split = forced;
     p.split = split;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];

@@ -60,6 +60,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "../../include/mq.h"
 #include "mq_debug.cuh"
 #include "mq_internal.h"
 #include "mq_nvfp4.cuh"
@@ -832,13 +833,6 @@ MQ_DEBUG_READER(debug_hits_gemm)
 }  // namespace gemm
 
 // ---------------------------------------------------------------- host side
-static int env_int(const char* name, int lo, int hi, int dflt) {
-    const char* v = getenv(name);
-    if (!v) return dflt;
-    const int x = atoi(v);
-    return (x >= lo && x <= hi) ? x : dflt;
-}
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1016,8 +1010,9 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.timeout = a.timeout_cycles;
     p.fault_skip_first_load = a.fault_skip_first_load;
     p.y_tma = y_tma ? 1 : 0;
-    p.group_m = env_int("MQ_GEMM_GROUP_M", 1, 1 << 20, GROUP_M);
-    p.stages = env_int("MQ_GEMM_STAGES", 2, C::STAGES, C::STAGES);
+    const int group_m = switch_value(MQ_SWITCH_GEMM_GROUP_M), stages = switch_value(MQ_SWITCH_GEMM_STAGES);
+    p.group_m = group_m > 0 ? group_m : GROUP_M;
+    p.stages = stages > 0 ? std::min(stages, C::STAGES) : C::STAGES;
     p.x = static_cast<const uint16_t*>(a.x);
     p.x_codes = const_cast<uint8_t*>(a.a_codes);
     p.x_scales = const_cast<uint8_t*>(a.a_scales);
@@ -1051,13 +1046,6 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kernel, ma, mb, my, msfb, msfa, p);
 }
 
-int env_choice(const char* name, int a, int b, int dflt) {
-    const char* v = getenv(name);
-    if (!v) return dflt;
-    const int x = atoi(v);
-    return (x == a || x == b) ? x : dflt;
-}
-
 }  // namespace
 
 int64_t fused_flag_count(int64_t M, int64_t K) {
@@ -1066,17 +1054,17 @@ int64_t fused_flag_count(int64_t M, int64_t K) {
 }
 
 // The 2-CTA form for M > 128, the 1-CTA form otherwise; the decode form for
-// M <= 64 (unfused).  MQ_GEMM_FORM=1|2 forces the prefill form and
-// MQ_GEMM_DECODE=0 keeps small M on the prefill kernel (the tests compare
-// the forms on the same shapes).
+// M <= 64 (unfused).  MQ_SWITCH_GEMM_FORM = 1 | 2 forces a prefill form and
+// MQ_SWITCH_GEMM_DECODE = 0 keeps small M on the prefill kernel (the tests
+// compare the forms on the same shapes).
 cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     if (a.swiglu_inter > 0) return launch_form<2, false, true>(a, num_sms, stream);
-    const char* dv = getenv("MQ_GEMM_DECODE");
-    if (!(dv && dv[0] == '0') && !getenv("MQ_GEMM_FORM") && !a.x && a.M <= 64) {
+    const int forced = switch_value(MQ_SWITCH_GEMM_FORM);
+    if (switch_value(MQ_SWITCH_GEMM_DECODE) == 1 && forced == 0 && !a.x && a.M <= 64) {
         const cudaError_t e = launch_gemm_decode(a, num_sms, stream);
         if (e != cudaErrorNotSupported) return e;
     }
-    const int form = env_choice("MQ_GEMM_FORM", 1, 2, a.M > gemm::BM ? 2 : 1);
+    const int form = forced != 0 ? forced : (a.M > gemm::BM ? 2 : 1);
     if (a.x) return form == 2 ? launch_form<2, true>(a, num_sms, stream) : launch_form<1, true>(a, num_sms, stream);
     return form == 2 ? launch_form<2, false>(a, num_sms, stream) : launch_form<1, false>(a, num_sms, stream);
 }

@@ -38,9 +38,13 @@ bool make_fp4_code_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int
 // MQ_ERR_SHAPE.
 int check_linear_shape(int64_t M, int64_t N, int64_t K);
 
+// The selectable alternatives of include/mq.h (MQ_SWITCH_*): the current
+// process-wide value of switch `which` (set from the environment on first use).
+int switch_value(int which);
+
 // Programmatic dependent launch: each kernel lets the next grid on the
 // stream launch early and waits (griddepcontrol.wait) before its first access
-// to global memory.  Launches carry the attribute unless MQ_PDL=0.
+// to global memory.  Launches carry the attribute unless MQ_SWITCH_PDL is 0.
 bool pdl_enabled();
 void set_pdl_attr(cudaLaunchAttribute* attr, int* nattr);
 

@@ -44,7 +44,20 @@ int scratch_for_current_device(void** addr) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+__global__ void k_fill_words(uint32_t* p, int n, uint32_t word) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = word;
+}
+
 }  // namespace
+
+extern "C" int mq_debug_noalloc_fill_header(uint32_t word, void* stream) {
+    void* scratch = nullptr;
+    const int st = scratch_for_current_device(&scratch);
+    if (st != MQ_OK) return st;
+    k_fill_words<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(scratch),
+                                                                   (int)(mq::WS_HEADER_BYTES / 4), word);
+    return cudaGetLastError() == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
+}
 
 extern "C" int mq_linear_w4a4_noalloc(const void* x, int64_t M, int64_t K, const uint8_t* w_codes,
                                       const uint8_t* w_scales, const float* alpha_w, int64_t N, void* y,

@@ -60,9 +60,13 @@ def lib() -> ctypes.CDLL:
         L.mq_mlp_w4a4.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, vp, vp, i64, vp, vp, sz, vp]
         L.mq_is_debug_build.argtypes = []
         L.mq_debug_bounds_hits.argtypes = [ctypes.POINTER(ctypes.c_int64)]
+        L.mq_set_switch.argtypes = [ctypes.c_int, ctypes.c_int]
+        L.mq_get_switch.argtypes = [ctypes.c_int]
+        L.mq_debug_noalloc_fill_header.argtypes = [ctypes.c_uint32, vp]
         for name in ("mq_tensor_scale", "mq_tensor_amax", "mq_alpha_from_amax", "mq_nvfp4_quantize",
                      "mq_nvfp4_gemm", "mq_linear_w4a4", "mq_read_status", "mq_nvfp4_gemm_swiglu",
-                     "mq_mlp_w4a4", "mq_is_debug_build", "mq_debug_bounds_hits"):
+                     "mq_mlp_w4a4", "mq_is_debug_build", "mq_debug_bounds_hits", "mq_set_switch",
+                     "mq_get_switch", "mq_debug_noalloc_fill_header"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -87,6 +91,52 @@ def _stream(stream):
 def _check(status: int, what: str):
     if status != MQ_OK:
         raise MQError(status, what)
+
+
+# -- selectable alternatives (MQ_SWITCH_* in mq.h) -------------------------
+
+SWITCHES = {"linear_path": 0, "gemm_form": 1, "gemm_decode": 2, "decode_split": 3, "gemm_stages": 4,
+            "gemm_group_m": 5, "pdl": 6}
+LINEAR_PATHS = {"onepass": 0, "split": 1, "ingemm": 2}
+
+
+def _switch_id(name) -> int:
+    return name if isinstance(name, int) else SWITCHES[name]
+
+
+def mq_set_switch(name, value: int) -> None:
+    """Set a process-wide switch by name (SWITCHES) or MQ_SWITCH_* number;
+    the linear path also takes its name (LINEAR_PATHS)."""
+    if name == "linear_path" and isinstance(value, str):
+        value = LINEAR_PATHS[value]
+    _check(lib().mq_set_switch(_switch_id(name), int(value)), f"mq_set_switch({name}, {value})")
+
+
+def mq_get_switch(name) -> int:
+    v = int(lib().mq_get_switch(_switch_id(name)))
+    if v < 0:
+        raise MQError(v, f"mq_get_switch({name})")
+    return v
+
+
+class switch:
+    """Context manager: `with mq.switch(gemm_form=2): ...` sets switches for
+    the block and puts the previous values back afterwards."""
+
+    def __init__(self, **values):
+        self.values = values
+        self.saved = {}
+
+    def __enter__(self):
+        for name, v in self.values.items():
+            self.saved[name] = mq_get_switch(name)
+            mq_set_switch(name, v)
+        return self
+
+    def __exit__(self, *exc):
+        for name, v in self.saved.items():
+            mq_set_switch(name, v)
+        return False
 
 
 # -- sizes ------------------------------------------------------------------

@@ -54,3 +54,19 @@ def brute(tmp_path_factory):
                                          ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32)]
     lib.brute_count_mismatch.restype = ctypes.c_uint64
     return lib
+
+
+@pytest.fixture
+def switches():
+    """Sets libmq's process-wide switches (mq.mq_set_switch) for one test and
+    restores every switch afterwards: `switches(gemm_form=2)`."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    saved = {name: mq.mq_get_switch(name) for name in mq.SWITCHES}
+
+    def set_(**values):
+        for name, v in values.items():
+            mq.mq_set_switch(name, v)
+
+    yield set_
+    for name, v in saved.items():
+        mq.mq_set_switch(name, v)

@@ -120,3 +120,31 @@ def test_debug_build_exports_the_same_symbols(libmq):
     dbg = ctypes.CDLL(build.DEBUG_LIB)
     assert dbg.mq_is_debug_build() == 1
     assert libmq.mq_is_debug_build() == 0
+
+
+def test_switches_without_gpu(libmq):
+    """The switch table answers on the host: defaults (or the environment's
+    values), range checks that keep the old value, and the numbering of
+    mq.h's MQ_SWITCH_* enumerators."""
+    from nvfp4_w4a4_quantized_03_b200 import mq
+    text = open(os.path.join(HEADER_DIR, "mq.h")).read()
+    enum = dict((k, int(v)) for k, v in re.findall(r"MQ_SWITCH_([A-Z_]+)\s*=\s*(\d+)", text))
+    assert enum.pop("COUNT") == len(mq.SWITCHES)
+    assert {k.lower(): v for k, v in enum.items()} == mq.SWITCHES
+    saved = {n: mq.mq_get_switch(n) for n in mq.SWITCHES}
+    try:
+        for name, good, bad in [("linear_path", 2, 3), ("gemm_form", 1, 3), ("gemm_decode", 0, 2),
+                                ("decode_split", 8, 3), ("gemm_stages", 2, 1), ("gemm_group_m", 7, -1),
+                                ("pdl", 0, 2)]:
+            mq.mq_set_switch(name, good)
+            assert mq.mq_get_switch(name) == good
+            assert libmq.mq_set_switch(mq.SWITCHES[name], bad) == -1       # MQ_ERR_INVALID_ARG
+            assert mq.mq_get_switch(name) == good
+        assert libmq.mq_get_switch(len(mq.SWITCHES)) == -1
+        assert libmq.mq_set_switch(-1, 0) == -1
+        with mq.switch(linear_path="split", gemm_form=2):
+            assert mq.mq_get_switch("linear_path") == 1 and mq.mq_get_switch("gemm_form") == 2
+        assert mq.mq_get_switch("linear_path") == 2 and mq.mq_get_switch("gemm_form") == 1
+    finally:
+        for n, v in saved.items():
+            mq.mq_set_switch(n, v)

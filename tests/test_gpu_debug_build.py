@@ -30,21 +30,18 @@ def _workloads():
         out += [q.codes.cpu().numpy(), q.scales.cpu().numpy()]
     for M, N, K, form in [(3, 17, 128, None), (64, 4096, 4096, None), (130, 300, 320, "1"), (257, 513, 1024, "2"),
                           (700, 1024, 4096, None)]:
-        if form:
-            os.environ["MQ_GEMM_FORM"] = form
         qx = mq.quantize(inputs.activation_bf16(M, K, seed=M, outlier_channels=3, device="cuda"))
         qw = mq.quantize(inputs.weight_bf16(N, K, seed=N, device="cuda"))
         y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-        mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, qw.codes, qw.scales, qw.alpha, M, N, K, y)
+        with mq.switch(gemm_form=int(form or 0)):
+            mq.mq_nvfp4_gemm(qx.codes, qx.scales, qx.alpha, qw.codes, qw.scales, qw.alpha, M, N, K, y)
         out.append(b16(y))
-        os.environ.pop("MQ_GEMM_FORM", None)
     M, K, N = 300, 1024, 768
     x = inputs.activation_bf16(M, K, seed=9, outlier_channels=10, device="cuda")
     lin = mq.LinearW4A4(inputs.weight_bf16(N, K, seed=10, device="cuda"))
     for path in ("onepass", "split", "ingemm"):
-        os.environ["MQ_LINEAR_PATH"] = path
-        out.append(b16(lin(x)))
-    os.environ.pop("MQ_LINEAR_PATH", None)
+        with mq.switch(linear_path=path):
+            out.append(b16(lin(x)))
     mlp = mq.MLPW4A4(inputs.weight_bf16(512, K, seed=11, device="cuda"), inputs.weight_bf16(384, 256, seed=12,
                                                                                          device="cuda"))
     out.append(b16(mlp(x)))

@@ -46,9 +46,9 @@ def _gemm(M, N, K, x, w):
 @pytest.mark.parametrize("M", [1, 2, 7, 16, 17, 33, 64])
 @pytest.mark.parametrize("N,K", [(4096, 4096), (130, 320), (6144, 4096), (300, 12288), (24576, 1024)])
 @pytest.mark.parametrize("split", ["auto", "1", "8"])
-def test_decode_gemm_against_oracle(M, N, K, split, monkeypatch):
+def test_decode_gemm_against_oracle(M, N, K, split, switches):
     if split != "auto":
-        monkeypatch.setenv("MQ_DECODE_SPLIT", split)
+        switches(decode_split=int(split))
     x = inputs.activation_bf16(M, K, seed=M * 7 + K, outlier_channels=max(1, inputs.outlier_count(K)),
                                outlier_scale=50.0)
     w = inputs.weight_bf16(N, K, seed=N + 3)
@@ -57,13 +57,13 @@ def test_decode_gemm_against_oracle(M, N, K, split, monkeypatch):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 12288, 4096), (64, 4096, 12288)])
-def test_decode_matches_prefill_kernel(M, N, K, monkeypatch):
+def test_decode_matches_prefill_kernel(M, N, K, switches):
     """The split-K kernel and the prefill-shaped kernel differ only in the
     order of the fp32 additions."""
     x = inputs.student_t_activation_bf16(M, K, seed=M + K)
     w = inputs.weight_bf16(N, K, seed=K + 1)
     a = _gemm(M, N, K, x, w)
-    monkeypatch.setenv("MQ_GEMM_DECODE", "0")
+    switches(gemm_decode=0)
     b = _gemm(M, N, K, x, w)
     assert rel_frobenius(bf16_bits_to_f64(a), bf16_bits_to_f64(b)) <= TOL
     _check_against_oracle(a, bits(x), bits(w))

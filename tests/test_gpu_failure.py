@@ -29,8 +29,8 @@ def _p(t):
 
 
 @pytest.mark.parametrize("form", ["1", "2"])
-def test_stalled_gemm_reports_timeout_and_context_survives(form, monkeypatch):
-    monkeypatch.setenv("MQ_GEMM_FORM", form)
+def test_stalled_gemm_reports_timeout_and_context_survives(form, switches):
+    switches(gemm_form=int(form))
     M, N, K = 256, 512, 1024
     x = inputs.activation_bf16(M, K, seed=9, outlier_channels=10).to(dev())
     w = inputs.weight_bf16(N, K, seed=10).to(dev())

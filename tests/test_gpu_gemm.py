@@ -23,11 +23,11 @@ TOL = 1e-3
 
 
 @pytest.fixture(params=["auto", "1", "2"])
-def gemm_form(request, monkeypatch):
+def gemm_form(request, switches):
     """Run a test with the library's choice of GEMM form, then forced to each
     of: one CTA (128 x 256 tiles) or a CTA pair (256 x 256 tiles)."""
     if request.param != "auto":
-        monkeypatch.setenv("MQ_GEMM_FORM", request.param)
+        switches(gemm_form=int(request.param))
     return request.param
 
 
@@ -146,13 +146,13 @@ def _check_linear_ws(ws, ref, M, K, rows=None):
 @pytest.mark.parametrize("M,N,K", [(1, 256, 64), (130, 300, 320), (257, 513, 1024), (700, 1024, 4096),
                                    (128, 256, 12288), (2100, 768, 2048)])
 @pytest.mark.parametrize("form", ["auto", "1", "2"])
-def test_linear_paths_agree(M, N, K, form, monkeypatch):
+def test_linear_paths_agree(M, N, K, form, switches):
     """The three ways mq_linear_w4a4 can quantize X -- the one-pass
     cooperative quantizer (default), the tensor-scale + quantize kernels, and
     quantizer warps inside the GEMM -- give the same Y bit for bit, and the
     oracle's within tolerance."""
     if form != "auto":
-        monkeypatch.setenv("MQ_GEMM_FORM", form)
+        switches(gemm_form=int(form))
     x, w = _random_case(M, N, K, seed=M + 3 * N + K, student_t=(M % 2 == 0))
     qw = mq.quantize(w.to(dev()))
     xd = x.to(dev())
@@ -160,7 +160,7 @@ def test_linear_paths_agree(M, N, K, form, monkeypatch):
     ref = oracle.linear_w4a4(bits(x), bits(w))
     outs = []
     for path in ("onepass", "split", "ingemm", "onepass"):
-        monkeypatch.setenv("MQ_LINEAR_PATH", path)
+        switches(linear_path=path)
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev())
         ws[linear_ws_offsets(M, K)[0]:].fill_(0x5A)      # stale bytes where the quantized activation goes
         mq.mq_linear_w4a4(xd, qw.codes, qw.scales, qw.alpha, N, y, ws)

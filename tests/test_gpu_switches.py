@@ -1,8 +1,9 @@
 """The GEMM's tuning switches give the default path's bytes: fewer pipeline
-stages (MQ_GEMM_STAGES), another tile raster (MQ_GEMM_GROUP_M), and launches
-without programmatic dependent launch (MQ_PDL=0, read once per process, so
-checked in a child process).  Codes, scales and Y are compared bit for bit
-with the default path on the same inputs."""
+stages (MQ_SWITCH_GEMM_STAGES), another tile raster (MQ_SWITCH_GEMM_GROUP_M)
+and launches without programmatic dependent launch (MQ_SWITCH_PDL = 0), set
+through mq_set_switch; and the environment sets a switch once, at the first
+call into the library (checked in a child process).  Codes, scales and Y are
+compared bit for bit with the default path on the same inputs."""
 import os
 import subprocess
 import sys
@@ -39,23 +40,28 @@ def default_result():
     return _run()
 
 
-@pytest.mark.parametrize("env", [{"MQ_GEMM_STAGES": "3"}, {"MQ_GEMM_STAGES": "2"},
-                                 {"MQ_GEMM_GROUP_M": "1"}, {"MQ_GEMM_GROUP_M": "5"}],
+@pytest.mark.parametrize("values", [{"gemm_stages": 3}, {"gemm_stages": 2}, {"gemm_group_m": 1},
+                                    {"gemm_group_m": 5}, {"pdl": 0}],
                          ids=lambda e: ",".join(f"{k}={v}" for k, v in e.items()))
-def test_switch_gives_the_default_bytes(env, default_result, monkeypatch):
-    for k, v in env.items():
-        monkeypatch.setenv(k, v)
+def test_switch_gives_the_default_bytes(values, default_result, switches):
+    switches(**values)
     got = _run()
     for a, b in zip(got, default_result):
         assert np.array_equal(a, b)
 
 
-def test_without_programmatic_dependent_launch(default_result, tmp_path):
+def test_environment_sets_a_switch_once(default_result, tmp_path):
+    """MQ_PDL=0 and MQ_GEMM_STAGES=3 in the environment of a fresh process
+    set the switches at the first call; changing the environment afterwards
+    changes nothing."""
     out = tmp_path / "y.npz"
-    code = ("import sys, numpy as np; sys.path.insert(0, %r); "
+    code = ("import os, sys, numpy as np; sys.path.insert(0, %r); "
+            "from nvfp4_w4a4_quantized_03_b200 import mq; "
+            "assert mq.mq_get_switch('pdl') == 0 and mq.mq_get_switch('gemm_stages') == 3; "
+            "os.environ['MQ_PDL'] = '1'; assert mq.mq_get_switch('pdl') == 0; "
             "from tests.test_gpu_switches import _run; r = _run(); "
             "np.savez(%r, *r)") % (ROOT, str(out))
-    env = dict(os.environ, MQ_PDL="0")
+    env = dict(os.environ, MQ_PDL="0", MQ_GEMM_STAGES="3")
     p = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert p.returncode == 0, p.stderr[-2000:]
     got = np.load(out)

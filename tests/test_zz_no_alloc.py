@@ -63,3 +63,25 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     dummy = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: the size check comes first
     st = f(dummy, M, K, dummy, dummy, dummy, N, dummy, None)
     assert st == -5, mq.lib().mq_status_string(st)      # MQ_ERR_WORKSPACE
+
+
+def test_noalloc_after_a_call_that_left_its_header_dirty():
+    """A call ended by a timeout can leave the scratch header's ticket, running
+    max, generation and status words nonzero; the next call clears the header
+    before its kernels run, so its output is the workspace entry point's."""
+    f = _noalloc_fn()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    M, K, N = 300, 2048, 512
+    w = inputs.weight_bf16(N, K, seed=23).to(dev())
+    qw = mq.quantize(w)
+    x = inputs.activation_bf16(M, K, seed=24, outlier_channels=20, outlier_scale=30.0).to(dev())
+    y_ref = torch.empty(M, N, dtype=torch.bfloat16, device=dev())
+    ws = mq.workspace(mq.mq_linear_w4a4_workspace_bytes(M, K), dev())
+    mq.mq_linear_w4a4(x, qw.codes, qw.scales, qw.alpha, N, y_ref, ws)
+    for word in (0xFFFFFFFF, 0x00000001, 0x7F7F0003):
+        assert mq.lib().mq_debug_noalloc_fill_header(word, stream) == 0
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev())
+        st = f(_p(x), M, K, _p(qw.codes), _p(qw.scales), _p(qw.alpha), N, _p(y), stream)
+        assert st == 0, mq.lib().mq_status_string(st)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(y), bits(y_ref)), hex(word)
