@@ -328,7 +328,8 @@ int mq_debug_noalloc_fill_header(uint32_t word, void *stream);
  *       0 every pipeline stage the prefill form has room for, else 2.. that
  *       many (fewer than the room are used as is).
  *   MQ_SWITCH_GEMM_GROUP_M  (MQ_GEMM_GROUP_M)
- *       0 the default tile raster (32 M-blocks per group), else 1 .. 2^20.
+ *       0 the tile raster by rule (groups of at most 32 M-blocks and 18 MiB
+ *       of A), else that many M-blocks per group, 1 .. 2^20.
  *   MQ_SWITCH_PDL           (MQ_PDL: 0 | 1)
  *       1 launches carry programmatic dependent launch (default), 0 not.
  *

@@ -82,7 +82,8 @@ constexpr int THREADS = (FIRST_EPI_WARP + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = BN;                     // stage st: SF_COL + st * SF_COLS_PER_STAGE
-constexpr int GROUP_M = 32;                         // tile raster: default M-blocks per group
+constexpr int GROUP_M = 32;                         // tile raster: at most this many M-blocks per group
+constexpr int64_t RASTER_A_BYTES = 18ll << 20;      // ... and at most this much of A (codes and scales)
 constexpr int MAX_STAGES = 10;
 constexpr int BARRIER_BYTES = 512;
 constexpr int SMEM_LIMIT = 232448;                  // dynamic shared memory per block on sm_100
@@ -1011,7 +1012,19 @@ cudaError_t launch_form(const GemmArgs& a, int num_sms, cudaStream_t stream) {
     p.fault_skip_first_load = a.fault_skip_first_load;
     p.y_tma = y_tma ? 1 : 0;
     const int group_m = switch_value(MQ_SWITCH_GEMM_GROUP_M), stages = switch_value(MQ_SWITCH_GEMM_STAGES);
-    p.group_m = group_m > 0 ? group_m : GROUP_M;
+    if (group_m > 0) {
+        p.group_m = group_m;
+    } else {
+        // Tiles walk N inside a group of M-blocks, so a group's rows of A are
+        // read from DRAM once if they stay in L2 while the group sweeps B, and
+        // B once per group.  32 M-blocks at K <= 4096 (the 8192-token set's
+        // whole A, 18 MB); at K = 12288 a group of 32 holds 54 MB of A, which
+        // was read ~2.3x from DRAM, so the group is cut to RASTER_A_BYTES
+        // (10 M-blocks there: DRAM reads 134 MB instead of 187 MB against
+        // 85 MB of A and B, and the launch no slower).
+        const int64_t a_block = (int64_t)C::TILE_M * (a.K / 2 + a.K / 16);
+        p.group_m = (int)std::max<int64_t>(4, std::min<int64_t>(GROUP_M, RASTER_A_BYTES / a_block));
+    }
     p.stages = stages > 0 ? std::min(stages, C::STAGES) : C::STAGES;
     p.x = static_cast<const uint16_t*>(a.x);
     p.x_codes = const_cast<uint8_t*>(a.a_codes);
