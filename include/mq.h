@@ -311,7 +311,7 @@ int mq_debug_noalloc_fill_header(uint32_t word, void *stream);
  * switch from its environment variable (named beside it), once; later
  * changes of the environment have no effect.
  *
- *   MQ_SWITCH_LINEAR_PATH   (MQ_LINEAR_PATH: onepass | split | ingemm)
+ *   MQ_SWITCH_LINEAR_PATH   (MQ_LINEAR_PATH: onepass | split | ingemm, or 0 | 1 | 2)
  *       how mq_linear_w4a4 quantizes X: 0 one cooperative kernel (amax, grid
  *       barrier, quantization; default), 1 the mq_tensor_scale and
  *       mq_nvfp4_quantize kernels, 2 the amax kernel and quantizer warps

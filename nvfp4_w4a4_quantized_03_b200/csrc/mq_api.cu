@@ -95,7 +95,8 @@ int switch_from_env(int which) {
     const SwitchDef& d = SWITCH_DEFS[which];
     const char* e = getenv(d.env);
     if (!e || !e[0]) return d.dflt;
-    if (which == MQ_SWITCH_LINEAR_PATH) return e[0] == 's' ? 1 : e[0] == 'i' ? 2 : 0;
+    if (which == MQ_SWITCH_LINEAR_PATH && !(e[0] >= '0' && e[0] <= '9'))
+        return e[0] == 's' ? 1 : e[0] == 'i' ? 2 : 0;            // onepass | split | ingemm
     const int v = atoi(e);
     return switch_value_ok(which, v) ? v : d.dflt;
 }

@@ -711,6 +711,16 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 // TMEM loads are double-buffered (chunk c + 1 loads while chunk
                 // c is scaled, rounded and staged); TMEM goes back to the MMA
                 // thread as soon as the last load has landed.
+                // Every CTA pair reaches its tile boundary at about the same
+                // time, and 16 boxes of Y per CTA leaving at once slow the next
+                // tile's first loads (clock64 traces: its third and fourth
+                // stages 1,000-2,000 cycles late).  So, except on the CTA's last
+                // tile (where a delay would only lengthen the launch), the
+                // epilogue warps space their stores over the next tile's first
+                // microseconds: warp w's first box after w x 200 ns, its second
+                // 1.6 us later (+2.6% on the four 8192-token projections,
+                // medians of 31 interleaved rounds; gate/up +4%).
+                const bool pace = tile + units < p.tiles;
                 uint8_t* box = epi_stage + (warp - FIRST_EPI_WARP) * C::EPI_BOX_BYTES;
                 const uint32_t box_row = smem_u32(box) + lane * 128;
                 const int row0 = mb * C::TILE_M + (int)rank * BM + quad * 32;
@@ -754,6 +764,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 __syncwarp();
                 if (lane == 0) arrive_leader<PAIR>(&s->acc_empty);
                 convert(rb, hi[1]);
+                if (pace && warp > FIRST_EPI_WARP) __nanosleep(200u * (uint32_t)(warp - FIRST_EPI_WARP));
+                __syncwarp();
                 issue(0);
                 if (lane == 0) bulk_wait_group_read0();
                 __syncwarp();
@@ -761,6 +773,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) stage_chunk(c * 4 + q, hi[c] + 4 * q);
+                if (pace) __nanosleep(1600u);
+                __syncwarp();
                 issue(1);
             } else if (!C::TMA_STORE && vec_ok && nb * BN + BN <= p.N) {
                 // Whole tile inside Y: drain this warp's 32 x 128 block of the

@@ -152,12 +152,15 @@ __device__ __forceinline__ void quantize_quad(int64_t rows, int64_t K, uint32_t 
 // the swizzle puts the 16-byte chunk j of row t at chunk j ^ (t % 8), so the
 // eight 16-byte shared-memory reads of a warp are conflict-free.  A ring of
 // QT_STAGES boxes per block keeps the loads in flight while earlier boxes are
-// quantized.  (Loading the same data with eight 16-byte global loads per
-// thread measured the L1 at 90% of its throughput, every warp-wide load
-// touching 32 cache lines, and ran 17-23% slower.)
+// quantized; two boxes per block let three blocks share an SM (the same
+// 192 KB in flight per SM as three boxes for two blocks, and half again as
+// many quantizing warps: the stand-alone quantize pass 2.5-3% faster).
+// (Loading the same data with eight 16-byte global loads per thread measured
+// the L1 at 90% of its throughput, every warp-wide load touching 32 cache
+// lines, and ran 17-23% slower.)
 constexpr int QT_THREADS = 256;
 constexpr int QT_ROWS = 256;
-constexpr int QT_STAGES = 3;
+constexpr int QT_STAGES = 2;
 constexpr int QT_BOX_BYTES = QT_ROWS * 128;
 constexpr int QT_SMEM = QT_STAGES * QT_BOX_BYTES + 1024;
 
@@ -173,7 +176,7 @@ constexpr int QT_SMEM = QT_STAGES * QT_BOX_BYTES + 1024;
 constexpr int QW_CONSUMERS = QT_THREADS / 32;
 constexpr int QW_THREADS = QT_THREADS + 32;
 
-__global__ void __launch_bounds__(QW_THREADS, 2)
+__global__ void __launch_bounds__(QW_THREADS, 3)
 k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
               const float* __restrict__ alpha_p, uint4* __restrict__ codes, uint8_t* __restrict__ scales) {
     extern __shared__ uint8_t smem_raw[];
@@ -246,7 +249,7 @@ k_quantize_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t pr
 // waits for another.  At the phase boundary the warps' maxima meet through an
 // mbarrier (one arrival per warp), thread 0 joins the grid barrier, and the
 // warps wait for alpha on a second mbarrier.  Every wait is bounded.
-__global__ void __launch_bounds__(QW_THREADS, 2)
+__global__ void __launch_bounds__(QW_THREADS, 3)
 k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, int64_t prows, int64_t K,
                       uint32_t* __restrict__ ws, float* __restrict__ alpha_out, uint4* __restrict__ codes,
                       uint8_t* __restrict__ scales, int* __restrict__ status, long long timeout) {
@@ -328,7 +331,7 @@ k_quantize_onepass_ws(const __grid_constant__ CUtensorMap xmap, int64_t rows, in
         fill_recip_table(rtab[warp], alpha, lane, 32);
         __syncwarp();
         qt.d = __fmul_rn(6.0f, alpha);
-            qt.rtab = rtab[warp];
+        qt.rtab = rtab[warp];
         ok = got && ok_shared != 0;
     };
     if (n == 0) boundary();

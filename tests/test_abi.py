@@ -148,3 +148,24 @@ def test_switches_without_gpu(libmq):
     finally:
         for n, v in saved.items():
             mq.mq_set_switch(n, v)
+
+
+def test_switches_read_from_the_environment_once(libmq):
+    """A fresh process takes each switch from its environment variable at the
+    first call (names or numbers for the linear path; invalid values keep the
+    default) and ignores later changes of the environment."""
+    import sys
+    code = ("import os, sys; sys.path.insert(0, %r); "
+            "from nvfp4_w4a4_quantized_03_b200 import mq; "
+            "print([mq.mq_get_switch(n) for n in ('linear_path', 'decode_split', 'gemm_stages', 'pdl', 'gemm_form')]); "
+            "os.environ['MQ_PDL'] = '1'; print(mq.mq_get_switch('pdl'))") % ROOT
+    env = dict(os.environ, MQ_LINEAR_PATH="ingemm", MQ_DECODE_SPLIT="3", MQ_GEMM_STAGES="1", MQ_PDL="0",
+               MQ_GEMM_FORM="2")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = out.stdout.split("\n")
+    assert lines[0] == "[2, 0, 0, 0, 2]", out.stdout
+    assert lines[1] == "0", out.stdout
+    env["MQ_LINEAR_PATH"] = "1"
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert out.stdout.split("\n")[0] == "[1, 0, 0, 0, 2]", out.stdout
