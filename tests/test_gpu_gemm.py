@@ -199,3 +199,27 @@ def test_prefill_projection_8k_sampled_rows(proj):
     _, err = check_gemm_elementwise(got, oracle.dequantize(xc_all[rows], xs_all[rows], ax),
                                     oracle.dequantize(wc, wsc, aw), K)
     assert err <= TOL
+
+
+def test_raster_groups_with_a_ragged_last_group(switches):
+    """At K = 16384 a raster group holds at most 18 MiB of A, i.e. 7 M-blocks
+    of 256 rows, so M = 2900 (12 M-blocks) runs as one group of 7 and a
+    ragged one of 5.  Every tile computes the same sums whatever the order of
+    the tiles: Y equals the one-M-block-per-group raster's bit for bit, and
+    the oracle on sampled rows within the per-element bound."""
+    M, N, K = 2900, 520, 16384
+    x, w = _random_case(M, N, K, seed=77)
+    ax, xc, xs, qx = gpu_quantize(x)
+    aw, wc, wsc, qw = gpu_quantize(w)
+    y = _gemm(qx, qw, M, N, K)
+    switches(gemm_group_m=1)
+    assert np.array_equal(_gemm(qx, qw, M, N, K), y)
+    rows = np.sort(np.random.default_rng(5).choice(M, 96, replace=False))
+    rows = np.union1d(rows, [0, 255, 256, 1791, 1792, 2899])          # group and block edges
+    assert oracle.tensor_scale(bits(x)) == ax and oracle.tensor_scale(bits(w)) == aw
+    x_codes, x_scales = oracle.quantize(bits(x)[rows], ax)
+    w_codes, w_scales = oracle.quantize(bits(w), aw)
+    assert np.array_equal(x_codes, xc[rows]) and np.array_equal(w_codes, wc)
+    _, err = check_gemm_elementwise(y[rows], oracle.dequantize(x_codes, x_scales, ax),
+                                    oracle.dequantize(w_codes, w_scales, aw), K)
+    assert err <= TOL, err
