@@ -163,12 +163,15 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                     // every wait on it runs out
                     skip = false;
                 } else {
-                    mbar_arrive_expect_tx(&s->ready[st], W_BYTES + p.MP * 128);
-                    tma_load_2d(stage_w(st), &tmap_w, &s->ready[st], kt * 128, n0);
-                    tma_load_2d(stage_x(st), &tmap_x, &s->ready[st], kt * 128, 0);
+                    // the scale slices first: their path (copy, scale writers,
+                    // TMEM store) is the longer one to the stage's barrier
+                    // (decode figures 0.6-1.6% faster than codes first)
                     mbar_arrive_expect_tx(&s->sf_full[st], 2 * nkb * 512);
                     bulk_load(stage_sfw(st), p.w_scales + (wt * p.katoms + ka) * 512, nkb * 512, &s->sf_full[st]);
                     bulk_load(stage_sfx(st), p.x_scales + ka * 512, nkb * 512, &s->sf_full[st]);
+                    mbar_arrive_expect_tx(&s->ready[st], W_BYTES + p.MP * 128);
+                    tma_load_2d(stage_w(st), &tmap_w, &s->ready[st], kt * 128, n0);
+                    tma_load_2d(stage_x(st), &tmap_x, &s->ready[st], kt * 128, 0);
                     pending |= 1u << st;
                     pending_phase = (pending_phase & ~(1u << st)) | (phase << st);
                 }
@@ -178,7 +181,7 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 // the copies this thread issued land before the CTA releases
                 // its shared memory: a stage's scale copies complete its
                 // sf_full barrier by themselves, its code tiles (issued just
-                // before them) get a short grace period
+                // after them) get a short grace period
                 for (int i = 0; i < STAGES; ++i)
                     if (pending & (1u << i))
                         mbar_wait_bounded(&s->sf_full[i], (pending_phase >> i) & 1, p.timeout, nullptr);
@@ -189,28 +192,47 @@ k_gemm_decode(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int st = 0;
-            uint32_t phase = 0;
-            for (int kt = kt0; kt < kt1; ++kt) {
-                if (!mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag)) { raise(); break; }
-                tc_fence_after();
-                const int nkb = min(NKB, p.kblocks - kt * NKB);
-                const uint64_t wd = smem_desc(smem_u32(stage_w(st)), 16, 1024, 2);
-                const uint64_t xd = smem_desc(smem_u32(stage_x(st)), 16, 1024, 2);
-                const uint32_t sf = tmem + SF_COL + st * 32;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    const uint64_t step = (uint64_t)(kb * 32 >> 4);
-                    mma_mxf4nvf4(tmem, wd + step, xd + step, IDESC, sf + kb * 4, sf + 16 + kb * 4,
-                                 (kt != kt0 || kb != 0) ? 1u : 0u);
+        // The whole warp runs the loop (its state stays warp-uniform) and one
+        // elected lane issues; a full stage's four MMAs go out as
+        // straight-line code with their operands computed first (as in
+        // k_gemm, where a lone lane in a divergent branch took ~360 cycles
+        // per stage to issue instead of ~140).
+        const bool leader = elect_one();
+        int st = 0;
+        uint32_t phase = 0;
+        for (int kt = kt0; kt < kt1; ++kt) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s->ready[st], phase, p.timeout, abort_flag))) {
+                if (leader) raise();
+                break;
+            }
+            tc_fence_after();
+            const int nkb = min(NKB, p.kblocks - kt * NKB);
+            const uint64_t wd = smem_desc(smem_u32(stage_w(st)), 16, 1024, 2);
+            const uint64_t xd = smem_desc(smem_u32(stage_x(st)), 16, 1024, 2);
+            const uint32_t sf = tmem + SF_COL + st * 32;
+            const uint32_t acc0 = kt != kt0 ? 1u : 0u;
+            if (leader) {
+                if (nkb == NKB) {
+                    mma_mxf4nvf4(tmem, wd, xd, IDESC, sf, sf + 16, acc0);
+                    mma_mxf4nvf4(tmem, wd + 2, xd + 2, IDESC, sf + 4, sf + 20, 1u);
+                    mma_mxf4nvf4(tmem, wd + 4, xd + 4, IDESC, sf + 8, sf + 24, 1u);
+                    mma_mxf4nvf4(tmem, wd + 6, xd + 6, IDESC, sf + 12, sf + 28, 1u);
+                } else {
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        const uint64_t step = (uint64_t)(kb * 32 >> 4);
+                        mma_mxf4nvf4(tmem, wd + step, xd + step, IDESC, sf + kb * 4, sf + 16 + kb * 4,
+                                     kb != 0 ? 1u : acc0);
+                    }
                 }
                 mma_commit(&s->empty[st]);
-                if (++st == STAGES) { st = 0; phase ^= 1; }
             }
-            // the epilogue waits for this; after an abort it still arrives, once
-            // the MMAs issued so far are done
-            mma_commit(&s->acc_full);
+            __syncwarp();
+            if (++st == STAGES) { st = 0; phase ^= 1; }
         }
+        // the epilogue waits for this; after an abort it still arrives, once
+        // the MMAs issued so far are done
+        if (leader) mma_commit(&s->acc_full);
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ scale writers
         const int quad = warp & 3;
