@@ -307,9 +307,9 @@ int mq_debug_noalloc_fill_header(uint32_t word, void *stream);
  * shapes that compute the same result (the tests compare their outputs bit
  * for bit); the defaults are the fastest measured.  A switch is one
  * process-wide value: mq_set_switch takes effect for launches enqueued after
- * it returns, from any thread.  The first call into the library sets every
- * switch from its environment variable (named beside it), once; later
- * changes of the environment have no effect.
+ * it returns, from any thread.  The first call that enqueues work or reads
+ * or sets a switch sets every switch from its environment variable (named
+ * beside it), once; later changes of the environment have no effect.
  *
  *   MQ_SWITCH_LINEAR_PATH   (MQ_LINEAR_PATH: onepass | split | ingemm, or 0 | 1 | 2)
  *       how mq_linear_w4a4 quantizes X: 0 one cooperative kernel (amax, grid
