@@ -103,8 +103,9 @@ struct Cfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t SF_COLS_PER_STAGE = 12 * NKB;   // per MMA: A 4 columns, B 8 columns
     static constexpr uint32_t SFB_OFF = 4 * NKB;              // B scales after the A scales of a stage
-    // Y leaves through shared memory and TMA stores in the pair form: one
-    // 32-row x 64-column bf16 box (4 KB, 128-byte swizzle) per epilogue warp
+    // In the pair form Y leaves through shared memory: one 32-row x 64-column
+    // bf16 box (4 KB, 128-byte swizzle) per epilogue warp, written out by the
+    // warp's own stores (the SwiGLU form's H by TMA stores)
     static constexpr bool TMA_STORE = PAIR == 2;
     static constexpr int EPI_BOX_BYTES = 32 * 64 * 2;
     static constexpr int EPI_BYTES = TMA_STORE ? EPI_WARPS * EPI_BOX_BYTES : 0;
@@ -141,7 +142,7 @@ struct Params {
     int* status;
     long long timeout;
     int fault_skip_first_load;
-    int y_tma;               // pair form: Y is written by TMA stores (tmap_y is valid; needs N % 8 == 0)
+    int y_tma;               // pair form: Y leaves through staged boxes (tmap_y is valid; needs N % 8 == 0)
     int group_m;             // tile raster: M-blocks per group (tiles walk N inside a group)
     int stages;              // pipeline stages in use (2 .. Cfg::STAGES)
     const uint16_t* x;       // fused linear: bf16 activation [M, K]
@@ -706,19 +707,23 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 if (lane == 0 && hmax != 0) atomicMax(p.h_amax, hmax << 16);
             } else if (C::TMA_STORE && p.y_tma) {
                 // This warp's 32 x 128 block of the accumulator leaves as two
-                // 32 x 64 bf16 boxes through the warp's staging buffer (TMA
-                // stores clip rows >= M and columns >= N).  The four 32-column
-                // TMEM loads are double-buffered (chunk c + 1 loads while chunk
-                // c is scaled, rounded and staged); TMEM goes back to the MMA
-                // thread as soon as the last load has landed.
+                // 32 x 64 bf16 boxes through the warp's staging buffer.  The
+                // four 32-column TMEM loads are double-buffered (chunk c + 1
+                // loads while chunk c is scaled, rounded and staged); TMEM goes
+                // back to the MMA thread as soon as the last load has landed.
+                // A staged box leaves through the warp's own 16-byte global
+                // stores, 8 lanes per 128-byte row and 4 rows per instruction
+                // (rows >= M and columns >= N skipped), not through a TMA
+                // store: the SM's TMA unit also issues the producer's loads,
+                // and 16 store boxes per CTA and tile queued in it delayed the
+                // next tile's first stages (the launch 2.5% faster; leaving
+                // Y out altogether, a timing-only copy, gained 4%).
                 // Every CTA pair reaches its tile boundary at about the same
-                // time, and 16 boxes of Y per CTA leaving at once slow the next
-                // tile's first loads (clock64 traces: its third and fourth
-                // stages 1,000-2,000 cycles late).  So, except on the CTA's last
-                // tile (where a delay would only lengthen the launch), the
-                // epilogue warps space their stores over the next tile's first
-                // microseconds: warp w's first box after w x 200 ns, its second
-                // 1.6 us later (+2.6% on the four 8192-token projections,
+                // time, so, except on the CTA's last tile (where a delay would
+                // only lengthen the launch), the epilogue warps also space
+                // their stores over the next tile's first microseconds: warp
+                // w's first box after w x 200 ns, its second 1.6 us later
+                // (+2.6% on the four 8192-token projections with TMA stores,
                 // medians of 31 interleaved rounds; gate/up +4%).
                 const bool pace = tile + units < p.tiles;
                 uint8_t* box = epi_stage + (warp - FIRST_EPI_WARP) * C::EPI_BOX_BYTES;
@@ -729,12 +734,17 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                     st_shared_v4(box_row + ((j ^ (lane & 7)) << 4), v[0], v[1], v[2], v[3]);
                 };
                 auto issue = [&](int h) {
-                    fence_proxy_async_shared();
-                    __syncwarp();
-                    if (lane == 0 && row0 < p.M && colh + h * 64 < p.N && MQ_CHECK_TMA_STORE(colh + h * 64, row0, 2)) {
-                        tma_store_2d(&tmap_y, box, colh + h * 64, row0);
-                        bulk_commit_group();
+                    __syncwarp();                               // the box is staged
+                    const int col = colh + h * 64 + (lane & 7) * 8;
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int r = it * 4 + (lane >> 3);
+                        const uint4 v = ld_shared_v4(smem_u32(box) + r * 128 + (((lane & 7) ^ (r & 7)) << 4));
+                        const int grow = row0 + r;
+                        if (grow < p.M && col < p.N && MQ_CHECK((int64_t)grow * p.N + col + 8 <= (int64_t)p.M * p.N))
+                            *reinterpret_cast<uint4*>(p.y + (int64_t)grow * p.N + col) = v;
                     }
+                    __syncwarp();                               // the box may be staged again
                 };
                 auto convert = [&](const uint32_t (&r)[32], uint32_t (&pk)[16]) {
 #pragma unroll
@@ -742,8 +752,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                         pk[j] = cvt_bf16x2(__fmul_rn(__uint_as_float(r[2 * j + 1]), ab),
                                            __fmul_rn(__uint_as_float(r[2 * j]), ab));
                 };
-                if (lane == 0) bulk_wait_group_read0();         // the previous tile's box has been read
-                __syncwarp();
                 uint32_t ra[32], rb[32], pk[16], hi[2][16];
                 tmem_ld_32x32b_x32(taddr, ra);
                 tmem_ld_wait_regs(ra);
@@ -767,8 +775,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUten
                 if (pace && warp > FIRST_EPI_WARP) __nanosleep(200u * (uint32_t)(warp - FIRST_EPI_WARP));
                 __syncwarp();
                 issue(0);
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
